@@ -1,0 +1,402 @@
+#!/usr/bin/env python
+"""Benchmark of the weight-only low-bit GEMM library on B200.
+
+Default workload: one denoise step of the FLUX.2-Klein-4B transformer's low-bit linear chain at
+a 1024x1024 image (4096 image + 512 text tokens): 5 double-stream blocks (image and text QKV,
+out, MLP-up, MLP-down) and 20 single-stream blocks (fused QKV+MLP-in, fused out), ternary
+2-bit weights with fp16 scales per group of 128, d = 3072. One step = one lowbit_gemm_batch
+call over the 80 linears, with inputs resident in HBM (3.7 GB of activations and 0.75 GB of
+packed weights, far larger than L2, so no flush is needed between steps).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl lowbit|reference]
+
+Prints one JSON line (rank 0). Under torchrun each rank runs its own replica (weak scaling);
+the timed region is bracketed by a barrier and a device synchronize and the max over ranks is
+reported. `--impl reference` times the CPU oracle (fp64, host cores) on a bounded sample of
+the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "low-bit GEMM TFLOP/s (% of B200 bf16 TC peak) at 1024² Klein shapes; HBM GB/s"
+UNIT = "TFLOP/s"
+DEFAULT_WORKLOAD = "klein_step_chain_1024sq_ternary_g128"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# --------------------------------------------------------------------------------------------
+# clocks sampled during the timed region
+# --------------------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", str(self.idx)], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for name, v in zip(names, r[5:9]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# --------------------------------------------------------------------------------------------
+# workload setup
+# --------------------------------------------------------------------------------------------
+def setup(specs, device, lb, torch, pinned=True):
+    """Device inputs / outputs for every linear (weights packed on the GPU by the library),
+    plus pinned host copies of the activations and host buffers for the outputs."""
+    items = []
+    for spec in specs:
+        prob = synth.make_problem(spec)
+        codes = torch.from_numpy(prob.codes).to(device)
+        packed = lb.pack(codes, spec.bits)
+        del codes
+        x_host = torch.from_numpy(prob.x_bf16.view(np.int16)).view(torch.bfloat16)
+        if pinned:
+            x_host = x_host.pin_memory()
+        x = x_host.to(device)
+        s = torch.from_numpy(prob.scales).to(device)
+        z = torch.from_numpy(prob.zeros).to(device) if prob.zeros is not None else None
+        y = torch.empty((spec.M, spec.N), dtype=torch.bfloat16, device=device)
+        y_host = torch.empty((spec.M, spec.N), dtype=torch.bfloat16, pin_memory=pinned)
+        items.append(dict(spec=spec, x=x, packed=packed, s=s, z=z, y=y, x_host=x_host, y_host=y_host))
+    descs = [lb.make_desc(it["x"], it["packed"], it["s"], it["z"], it["y"], it["spec"].bits,
+                          it["spec"].group_size) for it in items]
+    return items, descs
+
+
+def step_flops(specs):
+    return sum(s.flops for s in specs)
+
+
+def step_bytes(specs):
+    return sum(s.algorithmic_bytes() for s in specs)
+
+
+# --------------------------------------------------------------------------------------------
+# CPU oracle timing (bounded sample)
+# --------------------------------------------------------------------------------------------
+def oracle_sample(specs, rows_per_shape: int):
+    """Distinct shapes of the workload, each with its first `rows_per_shape` activation rows."""
+    seen = {}
+    for s in specs:
+        seen.setdefault((s.M, s.K, s.N, s.bits, s.group_size), s)
+    out = []
+    for s in seen.values():
+        prob = synth.make_problem(s)
+        m = min(rows_per_shape, s.M)
+        import oracle
+        packed, _ = oracle.pack(prob.codes, s.bits)
+        out.append((s, np.ascontiguousarray(prob.x_bf16[:m]), packed, prob.scales, prob.zeros, m))
+    return out
+
+
+def time_oracle(sample, threads=0):
+    import oracle
+    t0 = time.perf_counter()
+    flops = 0
+    for s, x, packed, sc, z, m in sample:
+        oracle.gemm(x, packed, sc, z, s.N, s.bits, s.group_size, threads=threads)
+        flops += 2 * m * s.K * s.N
+    dt = time.perf_counter() - t0
+    return flops, dt
+
+
+def cpu_baseline(specs, rows_per_shape=32):
+    import oracle
+    sample = oracle_sample(specs, rows_per_shape)
+    flops, dt = time_oracle(sample)
+    nshapes = len(sample)
+    return {"value": flops / dt / 1e12, "unit": UNIT, "cores": oracle.default().threads(0), "kind": "oracle",
+            "sample": f"{nshapes} distinct shapes of the workload, first {rows_per_shape} activation rows each "
+                      f"(full K and N, weights decoded inside the timed call); {flops / 1e9:.1f} GFLOP in {dt:.1f} s",
+            "host_cpus": os.cpu_count()}
+
+
+# --------------------------------------------------------------------------------------------
+# arms
+# --------------------------------------------------------------------------------------------
+def run_reference(args, specs, workload):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    rows = args.ref_rows
+    sample = oracle_sample(specs, rows)
+    for _ in range(args.warmup):
+        time_oracle(sample)
+    times = []
+    flops = 0
+    for _ in range(args.steps):
+        f, dt = time_oracle(sample)
+        flops = f
+        times.append(dt)
+    t = sum(times)
+    value = flops * args.steps / t / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * t / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": workload, "sample_rows_per_shape": rows},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.default().threads(0), "kind": "oracle",
+                             "sample": f"{len(sample)} distinct shapes, first {rows} activation rows each, "
+                                       f"{flops / 1e9:.1f} GFLOP per step"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_lowbit(args, specs, workload):
+    import torch
+    import torch.distributed as dist
+    import bit_weight_only_w2_b200 as lb
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        from datetime import timedelta
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local_rank))
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    lb.load()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(specs, args.ref_rows)   # before any timed GPU work; uses host cores only
+
+    items, descs = setup(specs, device, lb, torch, pinned=not args.no_e2e)
+    flops = step_flops(specs)
+    nbytes = step_bytes(specs)
+    stream = torch.cuda.current_stream(device)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # single-linear workloads fit in L2: flush it (write a buffer larger than L2) between steps
+    l2_bytes = torch.cuda.get_device_properties(device).L2_cache_size
+    need_flush = nbytes < 2 * l2_bytes
+    flush = torch.empty(int(max(2 * l2_bytes, 256 << 20)), dtype=torch.uint8, device=device) if need_flush else None
+
+    def one_step():
+        lb.gemm_batch(descs, device)
+
+    for _ in range(args.warmup):
+        one_step()
+    torch.cuda.synchronize(device)
+    if lb.device_status() != 0:
+        raise RuntimeError("kernel timeout reported during warm-up")
+
+    clocks = ClockSampler(device.index if device.index is not None else 0)
+    clocks.start()
+    barrier()
+    torch.cuda.synchronize(device)
+    if need_flush:
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        for a, b in evs:
+            flush.zero_()
+            a.record(stream)
+            one_step()
+            b.record(stream)
+        torch.cuda.synchronize(device)
+        ms_total = sum(a.elapsed_time(b) for a, b in evs)
+    else:
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            one_step()
+        b.record(stream)
+        torch.cuda.synchronize(device)
+        ms_total = a.elapsed_time(b)
+    barrier()
+    clk = clocks.stop()
+    ms_total = max_over_ranks(ms_total)
+    ms_step = ms_total / args.steps
+    value = world * flops / (ms_step * 1e-3) / 1e12
+    if lb.device_status() != 0:
+        raise RuntimeError("kernel timeout reported during the timed steps")
+
+    # per-launch durations of the (single) GEMM kernel, for the roofline: each linear timed on
+    # the launching stream with its own events, over two passes
+    per = []
+    for _ in range(2):
+        evs = []
+        for it in items:
+            if need_flush:
+                flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            lb.gemm(it["x"], it["packed"], it["s"], it["z"], it["spec"].bits, it["spec"].group_size, out=it["y"])
+            e1.record(stream)
+            evs.append((it["spec"], e0, e1))
+        torch.cuda.synchronize(device)
+        per.extend((sp, e0.elapsed_time(e1)) for sp, e0, e1 in evs)
+    launch_ms = sum(ms for _, ms in per) / len(per)
+    launch_flops = sum(sp.flops for sp, _ in per) / len(per)
+    launch_bytes = sum(sp.algorithmic_bytes() for sp, _ in per) / len(per)
+
+    # end to end: host activations -> device, the batch, outputs -> host, every step
+    e2e = None
+    if not args.no_e2e:
+        h2d = sum(it["x"].numel() * 2 for it in items)
+        d2h = sum(it["y"].numel() * 2 for it in items)
+        for _ in range(1):
+            for it in items:
+                it["x"].copy_(it["x_host"], non_blocking=True)
+            one_step()
+            for it in items:
+                it["y_host"].copy_(it["y"], non_blocking=True)
+        torch.cuda.synchronize(device)
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e2e_steps = max(1, min(args.steps, 5))
+        a.record(stream)
+        for _ in range(e2e_steps):
+            for it in items:
+                it["x"].copy_(it["x_host"], non_blocking=True)
+            one_step()
+            for it in items:
+                it["y_host"].copy_(it["y"], non_blocking=True)
+        b.record(stream)
+        torch.cuda.synchronize(device)
+        e2e_ms = max_over_ranks(a.elapsed_time(b)) / e2e_steps
+        e2e = {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_steps}
+
+    peaks, peak_src = load_peaks()
+    long_step = ms_step >= 5.0
+    peak_tf = peaks.get("bf16_tflops_sustained" if long_step else "bf16_tflops")
+    achieved = launch_flops / (launch_ms * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
+                "frac": achieved / peak_tf, "traffic": None,
+                "peak_source": f"{peak_src} {'sustained' if long_step else 'burst'} bf16 dense",
+                "kernel": "lowbit_gemm_kernel", "launches_timed": len(per),
+                "algorithmic_gflop_per_launch": launch_flops / 1e9,
+                "algorithmic_mb_per_launch": launch_bytes / 1e6,
+                "frac_of_burst_peak": achieved / peaks.get("bf16_tflops", peak_tf)}
+
+    if rank == 0:
+        spec0 = specs[0]
+        cfg = {"workload": workload, "linears_per_step": len(specs), "bits": spec0.bits,
+               "group_size": spec0.group_size, "gflop_per_step": flops / 1e9,
+               "algorithmic_mb_per_step": nbytes / 1e6,
+               "shapes_MKN": sorted({(s.M, s.K, s.N) for s in specs}),
+               "l2": "flushed between steps (256+ MB write)" if need_flush else "inputs larger than L2 (no flush)",
+               "parallelism": "replicas" if world > 1 else "single GPU"}
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
+                "hbm_gbs": world * nbytes / (ms_step * 1e-3) / 1e9,
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": len(specs) * args.steps, "clocks": clk}
+        print(json.dumps(line), flush=True)
+        if args.per_shape:
+            agg = {}
+            for sp, ms in per:
+                k = (sp.M, sp.K, sp.N)
+                agg.setdefault(k, []).append(ms)
+            for k, v in sorted(agg.items()):
+                m, kk, n = k
+                t = statistics.median(v)
+                print(f"# shape M={m} K={kk} N={n}: {t * 1e3:.1f} us, {2 * m * kk * n / t / 1e9:.1f} TFLOP/s",
+                      file=sys.stderr)
+    del items, descs
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="lowbit", choices=["lowbit", "reference"])
+    ap.add_argument("--ref-rows", type=int, default=32, help="activation rows per shape in the CPU oracle sample")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--per-shape", action="store_true", help="print per-shape launch times to stderr")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)   # at least 3 untimed warm-up steps
+    specs = synth.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, specs, args.workload)
+    return run_lowbit(args, specs, args.workload)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

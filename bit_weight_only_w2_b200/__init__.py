@@ -1,0 +1,170 @@
+"""Python binding of liblowbit.so: weight-only low-bit GEMM for B200 (sm_100a).
+
+Argument marshalling only: every step of the computation runs in the library's CUDA
+kernels. PyTorch provides device memory and streams. The binding raises if the library
+is missing; there is no fallback.
+
+    Y = gemm(x, packed, scales, zeros, bits, group_size)   # Y[M][N] = X[M][K] W^T
+
+Layouts (see include/lowbit.h): x bf16 [M][K]; packed int32 view of uint32 words
+[N][K*bits/32]; scales / zeros fp16 [K/group_size][N]; y bf16 [M][N].
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblowbit.so")
+
+STATUS = {
+    0: "LOWBIT_OK", 1: "LOWBIT_ERR_INVALID_ARG", 2: "LOWBIT_ERR_ALIGNMENT", 3: "LOWBIT_ERR_UNSUPPORTED",
+    4: "LOWBIT_ERR_UNSUPPORTED_DEVICE", 5: "LOWBIT_ERR_BAD_CODE", 6: "LOWBIT_ERR_TIMEOUT", 7: "LOWBIT_ERR_CUDA",
+}
+
+
+class LowbitError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS.get(status, status)}")
+
+
+class GemmDesc(ctypes.Structure):
+    _fields_ = [("M", ctypes.c_int64), ("N", ctypes.c_int64), ("K", ctypes.c_int64),
+                ("bits", ctypes.c_int), ("group_size", ctypes.c_int),
+                ("X", ctypes.c_void_p), ("Wp", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("zeros", ctypes.c_void_p), ("Y", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load liblowbit.so (raises FileNotFoundError if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise FileNotFoundError(f"{path} is missing: build it with `python -m bit_weight_only_w2_b200.build`")
+    lib = ctypes.CDLL(path)
+    i64, i32, p = ctypes.c_int64, ctypes.c_int, ctypes.c_void_p
+    lib.lowbit_status_string.argtypes = [i32]
+    lib.lowbit_status_string.restype = ctypes.c_char_p
+    lib.lowbit_version.restype = i32
+    lib.lowbit_packed_words.argtypes = [i64, i64, i32]
+    lib.lowbit_packed_words.restype = ctypes.c_size_t
+    lib.lowbit_pack.argtypes = [p, i64, i64, i32, p, p]
+    lib.lowbit_pack.restype = i32
+    lib.lowbit_unpack.argtypes = [p, i64, i64, i32, p, p]
+    lib.lowbit_unpack.restype = i32
+    lib.lowbit_gemm.argtypes = [i64, i64, i64, i32, i32, p, p, p, p, p, p]
+    lib.lowbit_gemm.restype = i32
+    lib.lowbit_gemm_ex.argtypes = [i64, i64, i64, i32, i32, p, p, p, p, p, i32, i32, p]
+    lib.lowbit_gemm_ex.restype = i32
+    lib.lowbit_gemm_batch.argtypes = [ctypes.POINTER(GemmDesc), i32, p]
+    lib.lowbit_gemm_batch.restype = i32
+    lib.lowbit_device_status.argtypes = [i32]
+    lib.lowbit_device_status.restype = i32
+    lib.lowbit_selftest_bounded_wait.argtypes = [ctypes.c_longlong, p]
+    lib.lowbit_selftest_bounded_wait.restype = i32
+    _lib = lib
+    return lib
+
+
+def _check(st: int, what: str) -> None:
+    if st != 0:
+        raise LowbitError(st, what)
+
+
+def _stream(t: Optional[torch.Tensor] = None) -> int:
+    dev = t.device if t is not None else None
+    return torch.cuda.current_stream(dev).cuda_stream
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _need(t: torch.Tensor, dtype, name: str):
+    if not t.is_cuda or t.dtype != dtype or not t.is_contiguous():
+        raise ValueError(f"{name}: expected a contiguous CUDA {dtype} tensor, got {t.dtype} on {t.device}")
+
+
+def version() -> int:
+    return int(load().lowbit_version())
+
+
+def packed_words(N: int, K: int, bits: int) -> int:
+    return int(load().lowbit_packed_words(N, K, bits))
+
+
+def pack(codes: torch.Tensor, bits: int) -> torch.Tensor:
+    """int8 codes [N][K] (binary -1/+1, ternary -1/0/+1, uint4 0..15) -> packed words
+    [N][K*bits/32] (int32 storage of uint32 words). Synchronous."""
+    _need(codes, torch.int8, "codes")
+    N, K = codes.shape
+    out = torch.empty((N, K * bits // 32), dtype=torch.int32, device=codes.device)
+    with torch.cuda.device(codes.device):
+        _check(load().lowbit_pack(_ptr(codes), N, K, bits, _ptr(out), _stream(codes)), "lowbit_pack")
+    return out
+
+
+def unpack(packed: torch.Tensor, N: int, K: int, bits: int) -> torch.Tensor:
+    _need(packed, torch.int32, "packed")
+    out = torch.empty((N, K), dtype=torch.int8, device=packed.device)
+    with torch.cuda.device(packed.device):
+        _check(load().lowbit_unpack(_ptr(packed), N, K, bits, _ptr(out), _stream(packed)), "lowbit_unpack")
+    return out
+
+
+def gemm(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, zeros: Optional[torch.Tensor],
+         bits: int, group_size: int, out: Optional[torch.Tensor] = None, tile_tokens: int = 0,
+         ksplit: int = 0) -> torch.Tensor:
+    """Y[M][N] = X[M][K] * W^T with W decoded from `packed`, `scales` (and `zeros`)."""
+    _need(x, torch.bfloat16, "x")
+    _need(packed, torch.int32, "packed")
+    _need(scales, torch.float16, "scales")
+    if zeros is not None:
+        _need(zeros, torch.float16, "zeros")
+    M, K = x.shape
+    N = scales.shape[1]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    else:
+        _need(out, torch.bfloat16, "out")
+    with torch.cuda.device(x.device):
+        lib = load()
+        if tile_tokens or ksplit:
+            st = lib.lowbit_gemm_ex(M, N, K, bits, group_size, _ptr(x), _ptr(packed), _ptr(scales), _ptr(zeros),
+                                    _ptr(out), tile_tokens, ksplit, _stream(x))
+        else:
+            st = lib.lowbit_gemm(M, N, K, bits, group_size, _ptr(x), _ptr(packed), _ptr(scales), _ptr(zeros),
+                                 _ptr(out), _stream(x))
+        _check(st, "lowbit_gemm")
+    return out
+
+
+def make_desc(x, packed, scales, zeros, y, bits: int, group_size: int) -> GemmDesc:
+    M, K = x.shape
+    N = scales.shape[1]
+    return GemmDesc(M, N, K, bits, group_size, _ptr(x), _ptr(packed), _ptr(scales), _ptr(zeros), _ptr(y))
+
+
+def gemm_batch(descs: Sequence[GemmDesc], device: Optional[torch.device] = None) -> None:
+    """Run the descriptors in order on the current stream (see lowbit_gemm_batch)."""
+    arr = (GemmDesc * len(descs))(*descs)
+    with torch.cuda.device(device if device is not None else torch.cuda.current_device()):
+        _check(load().lowbit_gemm_batch(arr, len(descs), _stream()), "lowbit_gemm_batch")
+
+
+def device_status(clear: bool = True) -> int:
+    """The device status word (0 = OK, LOWBIT_ERR_TIMEOUT if a kernel wait gave up)."""
+    return int(load().lowbit_device_status(1 if clear else 0))
+
+
+def selftest_bounded_wait(limit_cycles: int = 50_000_000) -> None:
+    """Launch the bounded-wait self-test kernel (see lowbit_selftest_bounded_wait)."""
+    _check(load().lowbit_selftest_bounded_wait(limit_cycles, _stream()), "lowbit_selftest_bounded_wait")

@@ -1,0 +1,665 @@
+// Weight-only low-bit GEMM for sm_100a:  Y[M][N] = X[M][K] * W^T,  W decoded from packed
+// binary / ternary / uint4 codes and fp16 group scales (and zeros).
+//
+// The multiply behind the Bonsai Image (FLUX.2-Klein-4B) transformer linears: binary weights
+// w = scale_g * b (bonsai-image-binary-4B-gemlite-1bit model card, "Binary Weight
+// Representation: 1-bit g128"), ternary 2-bit weights (mlx-vlm Bonsai article, model
+// overview) and the 4-bit group-64 text-encoder linears (same article, component
+// architecture). After decoding it is a dense contraction, so it runs on the tcgen05 tensor
+// cores.
+//
+// Kernel design ("swap AB", weights as the MMA's A operand):
+//   * One CTA tile = 128 weight rows (MMA M) x BT tokens (MMA N), K in stages of 128.
+//   * Warp 0 (one lane) is the TMA producer: per stage it loads two 64-wide, 128B-swizzled
+//     boxes of X (the MMA's B operand, K-major), the packed code box of the 128 rows and their
+//     group scales (and zeros) into a shared-memory ring.
+//   * The dequant warps each own 32 weight rows (one per lane, matching the tensor-memory lane
+//     quarter the warp may access): they read the row's packed words from shared memory,
+//     decode codes x scale to bf16 pairs with a few integer / bf16x2 instructions per pair,
+//     and store them straight into a tensor-memory ring with tcgen05.st. The decoded weights
+//     never touch shared memory, which leaves its bandwidth to TMA and the MMA's B reads.
+//   * Warp 1 (one lane) issues tcgen05.mma (kind::f16, A from tensor memory, B from shared
+//     memory, fp32 accumulators in tensor memory) and frees ring slots with tcgen05.commit.
+//   * Four epilogue warps read the accumulators with tcgen05.ld, round to bf16 and store Y.
+//     With two accumulator buffers the epilogue of one tile overlaps the next tile's MMAs.
+//   * Without split-K the grid is persistent (tiles strided over the CTAs). With split-K
+//     (small M, few tiles) the K range is divided over the CTAs of a thread-block cluster and
+//     the fp32 partial tiles are summed in a fixed order through distributed shared memory.
+//   * Every mbarrier wait is bounded (see sm100_ptx.cuh): a wait that gives up records
+//     LOWBIT_ERR_TIMEOUT in the device status word and the CTA drains and exits.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdint>
+#include <cstdio>
+
+#include "lowbit_internal.h"
+#include "sm100_ptx.cuh"
+
+namespace lowbit {
+
+__device__ unsigned g_device_status = 0;
+
+constexpr int kBlockN = 128;        // weight rows per tile (MMA M)
+constexpr int kBlockK = 128;        // K per pipeline stage
+constexpr int kNumCtrlWarps = 4;    // warp 0: TMA, warp 1: MMA + TMEM owner, warps 2-3 idle
+constexpr int kNumEpiWarps = 4;
+constexpr int kSmemLimit = 232448;  // 227 KB opt-in dynamic shared memory per block
+
+template <int BITS, int GS, int BT>
+struct Cfg {
+    static_assert(BITS == 1 || BITS == 2 || BITS == 4, "bits");
+    static_assert(GS == 64 || GS == 128, "group size");
+    static_assert(BT % 16 == 0 && BT >= 16 && BT <= 256, "MMA N");
+    static constexpr int kCtasPerSm = (BT <= 64) ? 2 : 1;
+    static constexpr int kNumDqWarps = (BITS == 4) ? 8 : 4;
+    static constexpr int kParts = kNumDqWarps / 4;                 // dequant warps per row quarter
+    static constexpr int kThreads = 32 * (kNumCtrlWarps + kNumEpiWarps + kNumDqWarps);
+    static constexpr int kFirstDqWarp = kNumCtrlWarps + kNumEpiWarps;
+    static constexpr int kNumAcc = (BT == 64 || BT == 256) ? 1 : 2;   // fit the tensor-memory budget
+    static constexpr int kAccCols = kNumAcc * BT;
+    static constexpr int kACol0 = (kAccCols + 31) / 32 * 32;
+    static constexpr int kNumA = (kCtasPerSm == 2) ? 3 : 4;          // A ring stages (64 columns each)
+    static constexpr int kColsUsed = kACol0 + kNumA * 64;
+    static constexpr int kTmemCols = kColsUsed <= 32 ? 32 : kColsUsed <= 64 ? 64 : kColsUsed <= 128 ? 128
+                                     : kColsUsed <= 256 ? 256 : 512;
+    static_assert(kColsUsed <= 512 && kTmemCols * kCtasPerSm <= 512, "tensor memory");
+
+    static constexpr int kWordsPerRow = kBlockK * BITS / 32;        // 4 / 8 / 16
+    static constexpr int kWRowBytes = kWordsPerRow * 4;             // 16 / 32 / 64
+    static constexpr int kXHalfBytes = BT * 128;                    // 64 bf16 per row
+    static constexpr int kXBytes = 2 * kXHalfBytes;
+    static constexpr int kWBytes = kBlockN * kWRowBytes;
+    static constexpr int kGroupsPerStage = kBlockK / GS;            // 1 or 2
+    static constexpr int kSBytes = kGroupsPerStage * kBlockN * 2;
+    static constexpr int kZBytes = (BITS == 4) ? kSBytes : 0;
+    static constexpr int kXOff = 0;
+    static constexpr int kWOff = kXBytes;
+    static constexpr int kSOff = kWOff + kWBytes;
+    static constexpr int kZOff = kSOff + kSBytes;
+    static constexpr int kStageBytes = (kZOff + kZBytes + 1023) / 1024 * 1024;
+    static constexpr int kTxBytes = kXBytes + kWBytes + kSBytes + kZBytes;
+    static constexpr int kBarBytes = 1024;
+    static constexpr int kBudget = kSmemLimit / kCtasPerSm - 1024 /*align*/ - kBarBytes - 2048 /*reserve*/;
+    static constexpr int kStagesFit = kBudget / kStageBytes;
+    static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
+    static_assert(kStages >= 2, "shared memory");
+    // Request enough shared memory that at most kCtasPerSm CTAs of these kernels share an SM:
+    // tensor memory (512 columns per SM) is not a scheduling resource, so residency is capped
+    // through shared memory instead (228 KB per SM).
+    static constexpr int kSmemNeeded = 1024 + kStages * kStageBytes + kBarBytes;
+    static constexpr int kSmemFloor = (kCtasPerSm == 2) ? 80 * 1024 : 150 * 1024;
+    static constexpr int kSmemBytes = kSmemNeeded > kSmemFloor ? kSmemNeeded : kSmemFloor;
+    static_assert(kSmemBytes <= kSmemLimit, "shared memory");
+    // split-K partial tile (fp32 [BT][128]) reuses the stage ring
+    static_assert(BT * kBlockN * 4 <= kStages * kStageBytes, "split-K partial buffer");
+    static constexpr uint32_t kIdesc = idesc_bf16_f32(kBlockN, BT);
+};
+
+struct KernelParams {
+    int M, N, K;
+    int num_kb;          // k-blocks of 128
+    int kb_per_split;    // k-blocks per cluster rank (split-K), else num_kb
+    int m_tiles, n_tiles, num_tiles;
+    int ksplit;          // cluster size along z (1 = persistent, no split)
+    __nv_bfloat16* Y;
+};
+
+// ---------------------------------------------------------------------------------------------
+// Decoders: one 64-wide K half of one weight row -> 32 bf16x2 values (even k low, odd k high).
+// ---------------------------------------------------------------------------------------------
+
+// Binary: bit 1 -> +s, 0 -> -s. Pair c of a word is (bit c, bit 16 + c); shifting the word
+// left by 15 - c puts them on the two bf16 sign bits, and one LOP3 flips the sign of s where
+// the bit is 0. Exact: the result is +-bf16(s).
+__device__ __forceinline__ void decode_half_b1(uint32_t w0, uint32_t w1, uint32_t s2, uint32_t (&out)[32]) {
+#pragma unroll
+    for (int c = 0; c < 16; ++c) out[c] = xor_andnot(s2, w0 << (15 - c), 0x80008000u);
+#pragma unroll
+    for (int c = 0; c < 16; ++c) out[16 + c] = xor_andnot(s2, w1 << (15 - c), 0x80008000u);
+}
+
+// Ternary: field f = t + 1 in {0,1,2}. OR-ing the two fields of a pair into the mantissas of
+// bf16 128.0 gives (128 + f * 4^j) exactly (j = field position inside the mantissa); one
+// bf16x2 FMA subtracts (128 + 4^j), leaving t * 4^j exactly, and a second multiplies by
+// s * 4^-j, giving t * s exactly (t in {-1,0,1}). s4[j] holds bf16x2(s * 4^-j).
+__device__ __forceinline__ void decode_word_b2(uint32_t v, const uint32_t (&s4)[3], uint32_t* out) {
+    constexpr uint32_t kMagic = 0x43004300u;                           // bf16x2(128, 128)
+    constexpr uint32_t kOne = 0x3F803F80u;                             // bf16x2(1, 1)
+    constexpr uint32_t kNegBase[3] = {0xC301C301u, 0xC304C304u, 0xC310C310u};  // -(128 + 4^j)
+    constexpr uint32_t kNegZero = 0x80008000u;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        const int shift = (c / 3) * 6;
+        const int j = c % 3;
+        const uint32_t e = and_or(v >> shift, 0x00030003u << (2 * j), kMagic);
+        const uint32_t t = bf16x2_fma(e, kOne, kNegBase[j]);
+        out[c] = bf16x2_fma(t, s4[j], kNegZero);
+    }
+}
+
+// uint4: OR-ing a nibble into bits 16..19 of fp32 128.0 gives 128 + q exactly; one FMA with
+// s and c = -(128 + z) * s gives (q - z) * s to fp32 rounding, then a pair is rounded to bf16.
+__device__ __forceinline__ void decode_word_b4(uint32_t v, float s, float cz, uint32_t* out) {
+    constexpr uint32_t kMagic = 0x43000000u;   // fp32 128.0
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        const uint32_t lo = and_or(v << (16 - 4 * c), 0x000F0000u, kMagic);
+        const uint32_t hi = and_or(v >> (4 * c), 0x000F0000u, kMagic);
+        out[c] = pack_bf16x2(fmaf(__uint_as_float(lo), s, cz), fmaf(__uint_as_float(hi), s, cz));
+    }
+}
+
+__device__ __forceinline__ uint32_t bf16x2_splat(float f) {
+    const __nv_bfloat16 b = __float2bfloat16_rn(f);
+    const uint32_t u = static_cast<uint32_t>(__bfloat16_as_ushort(b));
+    return u | (u << 16);
+}
+
+// ---------------------------------------------------------------------------------------------
+// The kernel
+// ---------------------------------------------------------------------------------------------
+template <int BITS, int GS, int BT>
+__global__ void __launch_bounds__(Cfg<BITS, GS, BT>::kThreads, Cfg<BITS, GS, BT>::kCtasPerSm)
+    lowbit_gemm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w,
+                       const __grid_constant__ CUtensorMap map_s, const __grid_constant__ CUtensorMap map_z,
+                       const KernelParams p) {
+    using C = Cfg<BITS, GS, BT>;
+    constexpr int S = C::kStages;
+    constexpr int NA = C::kNumA;
+    constexpr int NACC = C::kNumAcc;
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* bar_area = smem + S * C::kStageBytes;
+    uint64_t* full = reinterpret_cast<uint64_t*>(bar_area);
+    uint64_t* empty = full + S;
+    uint64_t* afull = empty + S;
+    uint64_t* aempty = afull + NA;
+    uint64_t* accfull = aempty + NA;
+    uint64_t* accempty = accfull + NACC;
+    uint64_t* drain = accempty + NACC;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < S; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], 1 + C::kNumDqWarps);
+        }
+        for (int i = 0; i < NA; ++i) {
+            mbar_init(&afull[i], C::kNumDqWarps);
+            mbar_init(&aempty[i], 1);
+        }
+        for (int i = 0; i < NACC; ++i) {
+            mbar_init(&accfull[i], 1);
+            mbar_init(&accempty[i], kNumEpiWarps);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&map_x);
+        tma_prefetch_desc(&map_w);
+        tma_prefetch_desc(&map_s);
+        if (BITS == 4) tma_prefetch_desc(&map_z);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_holder, C::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+
+    // Wait for the previous kernel in the stream (programmatic dependent launch), then let
+    // the next one start its prologue as soon as SMs free up.
+    grid_dependency_wait();
+    grid_launch_dependents();
+
+    const bool split = p.ksplit > 1;
+    const int kb_begin = split ? static_cast<int>(blockIdx.z) * p.kb_per_split : 0;
+    const int kb_end = split ? min(p.num_kb, kb_begin + p.kb_per_split) : p.num_kb;
+    const int tile_step = split ? p.num_tiles : static_cast<int>(gridDim.x);
+    unsigned* status = &g_device_status;
+
+    if (warp == 0) {
+        // ---------------------------------------------------------------- TMA producer
+        if (lane == 0) {
+            uint32_t it = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += tile_step) {
+                const int m0 = (tile / p.n_tiles) * BT;
+                const int n0 = (tile % p.n_tiles) * kBlockN;
+                for (int kb = kb_begin; kb < kb_end; ++kb, ++it) {
+                    const uint32_t s = it % S, ph = (it / S) & 1u;
+                    if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, status)) { ok = false; break; }
+                    uint8_t* st = smem + s * C::kStageBytes;
+                    mbar_arrive_expect_tx(&full[s], C::kTxBytes);
+                    tma_load_2d(&map_x, &full[s], st + C::kXOff, kb * kBlockK, m0);
+                    tma_load_2d(&map_x, &full[s], st + C::kXOff + C::kXHalfBytes, kb * kBlockK + 64, m0);
+                    tma_load_2d(&map_w, &full[s], st + C::kWOff, kb * C::kWordsPerRow, n0);
+                    tma_load_2d(&map_s, &full[s], st + C::kSOff, n0, kb * C::kGroupsPerStage);
+                    if (BITS == 4) tma_load_2d(&map_z, &full[s], st + C::kZOff, n0, kb * C::kGroupsPerStage);
+                }
+            }
+            if (!ok) {
+                // Drain: wait (bounded) for the copies still in flight before the CTA exits.
+                for (uint32_t j = (it > (uint32_t)S ? it - S : 0u); j < it; ++j) {
+                    const long long t0 = clock64();
+                    while (!mbar_try_wait(&full[j % S], (j / S) & 1u) && clock64() - t0 < kWaitLimitCycles) {
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            uint32_t it = 0, ait = 0, tcount = 0;
+            bool ok = true;
+            bool issued = false;
+            for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += tile_step, ++tcount) {
+                const uint32_t b = tcount % NACC, acc_ph = (tcount / NACC) & 1u;
+                if (!mbar_wait(&accempty[b], acc_ph ^ 1u, abort_flag, status)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + b * BT;
+                for (int kb = kb_begin; kb < kb_end; ++kb, ++it, ++ait) {
+                    const uint32_t s = it % S, ph = (it / S) & 1u;
+                    const uint32_t a = ait % NA, aph = (ait / NA) & 1u;
+                    if (!mbar_wait(&full[s], ph, abort_flag, status)) { ok = false; break; }
+                    if (!mbar_wait(&afull[a], aph, abort_flag, status)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t xs = smem_u32(smem + s * C::kStageBytes + C::kXOff);
+#pragma unroll
+                    for (int kk = 0; kk < kBlockK / 16; ++kk) {
+                        const uint32_t a_tmem = tmem_base + C::kACol0 + a * 64 + kk * 8;
+                        const uint64_t bdesc =
+                            smem_desc_k_sw128(xs + (kk >> 2) * C::kXHalfBytes + (kk & 3) * 32);
+                        mma_bf16_ts(d_tmem, a_tmem, bdesc, C::kIdesc, (kb > kb_begin || kk > 0) ? 1u : 0u);
+                    }
+                    issued = true;
+                    mma_commit(&empty[s]);
+                    mma_commit(&aempty[a]);
+                }
+                if (!ok) break;
+                mma_commit(&accfull[b]);
+            }
+            if (!ok && issued) {
+                // Drain: make sure no MMA is still writing tensor memory before it is freed.
+                mma_commit(drain);
+                const long long t0 = clock64();
+                while (!mbar_try_wait(drain, 0) && clock64() - t0 < kWaitLimitCycles) {
+                }
+            }
+        }
+    } else if (warp >= C::kFirstDqWarp) {
+        // ---------------------------------------------------------------- dequant warps
+        const int dq = warp - C::kFirstDqWarp;
+        const int quarter = warp & 3;
+        const int part = dq >> 2;                    // which K part of the stage this warp decodes
+        const int row = quarter * 32 + lane;         // weight row within the tile = TMEM lane
+        const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
+        constexpr int kHalvesPerPart = 2 / C::kParts;   // 64-wide K halves decoded by this warp
+        uint32_t it = 0, ait = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += tile_step) {
+            for (int kb = kb_begin; kb < kb_end; ++kb, ++it, ++ait) {
+                const uint32_t s = it % S, ph = (it / S) & 1u;
+                const uint32_t a = ait % NA, aph = (ait / NA) & 1u;
+                if (!__all_sync(0xffffffffu, mbar_wait(&full[s], ph, abort_flag, status))) { ok = false; break; }
+                const uint8_t* st = smem + s * C::kStageBytes;
+                // --- read this row's packed words and scales from shared memory
+                uint32_t words[kHalvesPerPart][C::kWordsPerRow / 2];
+                const uint8_t* wrow = st + C::kWOff + row * C::kWRowBytes;
+#pragma unroll
+                for (int hh = 0; hh < kHalvesPerPart; ++hh) {
+                    const int h = part * kHalvesPerPart + hh;
+                    if (BITS == 1) {
+                        const uint2 v = *reinterpret_cast<const uint2*>(wrow + h * 8);
+                        words[hh][0] = v.x;
+                        words[hh][1] = v.y;
+                    } else if (BITS == 2) {
+                        const int chunk = h ^ ((row >> 2) & 1);           // 32-byte swizzle
+                        const uint4 v = *reinterpret_cast<const uint4*>(wrow + chunk * 16);
+                        words[hh][0] = v.x; words[hh][1] = v.y; words[hh][2] = v.z; words[hh][3] = v.w;
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < 2; ++q) {
+                            const int chunk = (2 * h + q) ^ ((row >> 1) & 3);  // 64-byte swizzle
+                            const uint4 v = *reinterpret_cast<const uint4*>(wrow + chunk * 16);
+                            words[hh][4 * q + 0] = v.x; words[hh][4 * q + 1] = v.y;
+                            words[hh][4 * q + 2] = v.z; words[hh][4 * q + 3] = v.w;
+                        }
+                    }
+                }
+                float sc[kHalvesPerPart], zc[kHalvesPerPart];
+#pragma unroll
+                for (int hh = 0; hh < kHalvesPerPart; ++hh) {
+                    const int h = part * kHalvesPerPart + hh;
+                    const int gi = (GS == 64) ? h : 0;
+                    const __half* srow = reinterpret_cast<const __half*>(st + C::kSOff) + gi * kBlockN;
+                    sc[hh] = __half2float(srow[row]);
+                    if (BITS == 4) {
+                        const __half* zrow = reinterpret_cast<const __half*>(st + C::kZOff) + gi * kBlockN;
+                        zc[hh] = __half2float(zrow[row]);
+                    } else {
+                        zc[hh] = 0.f;
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[s]);
+                // --- decode into the tensor-memory A ring
+                if (!__all_sync(0xffffffffu, mbar_wait(&aempty[a], aph ^ 1u, abort_flag, status))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+#pragma unroll
+                for (int hh = 0; hh < kHalvesPerPart; ++hh) {
+                    const int h = part * kHalvesPerPart + hh;
+                    uint32_t out[32];
+                    if (BITS == 1) {
+                        decode_half_b1(words[hh][0], words[hh][1], bf16x2_splat(sc[hh]), out);
+                    } else if (BITS == 2) {
+                        const uint32_t s4[3] = {bf16x2_splat(sc[hh]), bf16x2_splat(sc[hh] * 0.25f),
+                                                bf16x2_splat(sc[hh] * 0.0625f)};
+#pragma unroll
+                        for (int w = 0; w < 4; ++w) decode_word_b2(words[hh][w], s4, out + 8 * w);
+                    } else {
+                        const float cz = -(128.0f + zc[hh]) * sc[hh];
+#pragma unroll
+                        for (int w = 0; w < 8; ++w) decode_word_b4(words[hh][w], sc[hh], cz, out + 4 * w);
+                    }
+                    tmem_st32(lane_base + C::kACol0 + a * 64 + h * 32, out);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&afull[a]);
+            }
+        }
+    } else if (warp >= kNumCtrlWarps && warp < kNumCtrlWarps + kNumEpiWarps) {
+        // ---------------------------------------------------------------- epilogue warps
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;
+        const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
+        uint32_t tcount = 0;
+        for (int tile = blockIdx.x; tile < p.num_tiles; tile += tile_step, ++tcount) {
+            const uint32_t b = tcount % NACC, acc_ph = (tcount / NACC) & 1u;
+            if (!__all_sync(0xffffffffu, mbar_wait(&accfull[b], acc_ph, abort_flag, status))) break;
+            tc_fence_after();
+            const int m0 = (tile / p.n_tiles) * BT;
+            const int n = (tile % p.n_tiles) * kBlockN + row;
+            constexpr int kChunk = (BT >= 32) ? 32 : 16;
+#pragma unroll 1
+            for (int c0 = 0; c0 < BT; c0 += kChunk) {
+                uint32_t v[32];
+                if (kChunk == 32) {
+                    tmem_ld32(lane_base + b * BT + c0, v);
+                } else {
+                    tmem_ld16(lane_base + b * BT + c0, *reinterpret_cast<uint32_t(*)[16]>(v));
+                }
+                tmem_wait_ld();
+                if (!split) {
+                    if (n < p.N) {
+#pragma unroll
+                        for (int j = 0; j < kChunk; ++j) {
+                            const int m = m0 + c0 + j;
+                            if (m < p.M)
+                                p.Y[static_cast<size_t>(m) * p.N + n] = __float2bfloat16_rn(__uint_as_float(v[j]));
+                        }
+                    }
+                } else {
+                    float* part = reinterpret_cast<float*>(smem);
+#pragma unroll
+                    for (int j = 0; j < kChunk; ++j) part[(c0 + j) * kBlockN + row] = __uint_as_float(v[j]);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&accempty[b]);
+        }
+    }
+
+    __syncwarp();
+    if (split) {
+        // Sum the K-slices of the cluster in rank order; rank r reduces columns c = r mod ksplit.
+        cluster_sync_all();
+        if (warp >= kNumCtrlWarps && warp < kNumCtrlWarps + kNumEpiWarps && !*abort_flag) {
+            const int row = (warp & 3) * 32 + lane;
+            const int tile = blockIdx.x;
+            const int m0 = (tile / p.n_tiles) * BT;
+            const int n = (tile % p.n_tiles) * kBlockN + row;
+            const uint32_t rank = cluster_ctarank();
+            const uint32_t part0 = smem_u32(smem);
+            if (n < p.N) {
+                for (int c = static_cast<int>(rank); c < BT; c += p.ksplit) {
+                    const int m = m0 + c;
+                    if (m >= p.M) break;
+                    const uint32_t off = static_cast<uint32_t>((c * kBlockN + row) * 4);
+                    float acc = 0.f;
+                    for (int q = 0; q < p.ksplit; ++q) acc += ld_shared_cluster_f32(map_shared_rank(part0 + off, q));
+                    p.Y[static_cast<size_t>(m) * p.N + n] = __float2bfloat16_rn(acc);
+                }
+            }
+        }
+        cluster_sync_all();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::kTmemCols);
+    }
+}
+
+// One CTA waits on a barrier that nothing arrives on, with the GEMM's bounded wait: the wait
+// gives up after `limit` clocks and records the timeout in the device status word.
+__global__ void bounded_wait_selftest_kernel(long long limit) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, &g_device_status, limit);
+}
+
+lowbit_status selftest_bounded_wait(long long limit_cycles, cudaStream_t stream) {
+    bounded_wait_selftest_kernel<<<1, 32, 0, stream>>>(limit_cycles);
+    return cudaGetLastError() == cudaSuccess ? LOWBIT_OK : LOWBIT_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------------------------
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        cudaDriverEntryPointQueryResult q;
+        void* f = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    }
+    return fn;
+}
+
+bool make_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, int elem_bytes, const void* base, uint64_t inner,
+                 uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                 CUtensorMapSwizzle swz) {
+    auto fn = get_encode_fn();
+    if (!fn) return false;
+    (void)elem_bytes;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {row_bytes};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+int num_sms() {
+    static int sms = 0;
+    if (!sms) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (sms <= 0) sms = 148;
+    }
+    return sms;
+}
+
+template <int BITS, int GS, int BT>
+lowbit_status launch(const GemmProblem& g, int ksplit_request, cudaStream_t stream) {
+    using C = Cfg<BITS, GS, BT>;
+    auto kernel = lowbit_gemm_kernel<BITS, GS, BT>;
+    static bool attr_done = false;
+    if (!attr_done) {
+        if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
+            return LOWBIT_ERR_CUDA;
+        attr_done = true;
+    }
+    CUtensorMap mx, mw, ms, mz;
+    const int K = static_cast<int>(g.K), N = static_cast<int>(g.N), M = static_cast<int>(g.M);
+    const CUtensorMapSwizzle wswz = C::kWRowBytes == 16   ? CU_TENSOR_MAP_SWIZZLE_NONE
+                                    : C::kWRowBytes == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                                          : CU_TENSOR_MAP_SWIZZLE_64B;
+    bool ok = make_map_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.X, K, M, uint64_t(K) * 2, 64, BT,
+                          CU_TENSOR_MAP_SWIZZLE_128B);
+    ok = ok && make_map_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, g.Wp, uint64_t(K) * BITS / 32, N,
+                           uint64_t(K) * BITS / 8, C::kWordsPerRow, kBlockN, wswz);
+    ok = ok && make_map_2d(&ms, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, g.scales, N, K / GS, uint64_t(N) * 2, kBlockN,
+                           C::kGroupsPerStage, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (BITS == 4)
+        ok = ok && make_map_2d(&mz, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, g.zeros, N, K / GS, uint64_t(N) * 2,
+                               kBlockN, C::kGroupsPerStage, CU_TENSOR_MAP_SWIZZLE_NONE);
+    else
+        mz = ms;
+    if (!ok) return LOWBIT_ERR_CUDA;
+
+    KernelParams p;
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.num_kb = (K + kBlockK - 1) / kBlockK;
+    p.m_tiles = (M + BT - 1) / BT;
+    p.n_tiles = (N + kBlockN - 1) / kBlockN;
+    p.num_tiles = p.m_tiles * p.n_tiles;
+    p.Y = static_cast<__nv_bfloat16*>(g.Y);
+    int ksplit = ksplit_request;
+    if (ksplit < 1) ksplit = 1;
+    if (ksplit > 8) ksplit = 8;
+    if (ksplit > p.num_kb) ksplit = p.num_kb;
+    int kbps = (p.num_kb + ksplit - 1) / ksplit;
+    ksplit = (p.num_kb + kbps - 1) / kbps;     // every rank gets at least one k-block
+    p.kb_per_split = ksplit > 1 ? kbps : p.num_kb;
+    p.ksplit = ksplit;
+
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attrs[2];
+    int na = 0;
+    attrs[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attrs[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+    if (ksplit > 1) {
+        cfg.gridDim = dim3(p.num_tiles, 1, ksplit);
+        attrs[na].id = cudaLaunchAttributeClusterDimension;
+        attrs[na].val.clusterDim.x = 1;
+        attrs[na].val.clusterDim.y = 1;
+        attrs[na].val.clusterDim.z = ksplit;
+        ++na;
+    } else {
+        const int slots = num_sms() * C::kCtasPerSm;
+        cfg.gridDim = dim3(p.num_tiles < slots ? p.num_tiles : slots, 1, 1);
+    }
+    cfg.blockDim = dim3(C::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = stream;
+    cfg.attrs = attrs;
+    cfg.numAttrs = na;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, mx, mw, ms, mz, p);
+    return e == cudaSuccess ? LOWBIT_OK : LOWBIT_ERR_CUDA;
+}
+
+// Token-tile width for M rows.
+int pick_bt(int64_t M) {
+    if (M <= 16) return 16;
+    if (M <= 32) return 32;
+    if (M <= 64) return 64;
+    if (M <= 128) return 128;
+    return 256;
+}
+
+int ctas_per_sm_for(int bt) { return bt <= 64 ? 2 : 1; }
+
+template <int BITS, int GS>
+lowbit_status launch_bits_gs(const GemmProblem& g, int bt, int ksplit, cudaStream_t s) {
+    switch (bt) {
+        case 16: return launch<BITS, GS, 16>(g, ksplit, s);
+        case 32: return launch<BITS, GS, 32>(g, ksplit, s);
+        case 64: return launch<BITS, GS, 64>(g, ksplit, s);
+        case 128: return launch<BITS, GS, 128>(g, ksplit, s);
+        case 256: return launch<BITS, GS, 256>(g, ksplit, s);
+        default: return LOWBIT_ERR_UNSUPPORTED;
+    }
+}
+
+}  // namespace
+
+// Chooses the tile width and split-K factor, then launches. `force_bt` / `force_split`
+// (0 = automatic) pin them for tests and tuning.
+lowbit_status gemm_launch(const GemmProblem& g, int force_bt, int force_split, cudaStream_t stream) {
+    const int bt = force_bt ? force_bt : pick_bt(g.M);
+    int ksplit = force_split;
+    if (!ksplit) {
+        const int64_t tiles = ((g.M + bt - 1) / bt) * ((g.N + kBlockN - 1) / kBlockN);
+        const int64_t slots = static_cast<int64_t>(num_sms()) * ctas_per_sm_for(bt);
+        const int64_t num_kb = (g.K + kBlockK - 1) / kBlockK;
+        ksplit = 1;
+        if (tiles * 2 <= slots && num_kb >= 4) {
+            int64_t s = slots / tiles;
+            if (s > 8) s = 8;
+            if (s > num_kb / 2) s = num_kb / 2;
+            ksplit = static_cast<int>(s < 1 ? 1 : s);
+        }
+    }
+    switch (g.bits * 1000 + g.group_size) {
+        case 1064: return launch_bits_gs<1, 64>(g, bt, ksplit, stream);
+        case 1128: return launch_bits_gs<1, 128>(g, bt, ksplit, stream);
+        case 2064: return launch_bits_gs<2, 64>(g, bt, ksplit, stream);
+        case 2128: return launch_bits_gs<2, 128>(g, bt, ksplit, stream);
+        case 4064: return launch_bits_gs<4, 64>(g, bt, ksplit, stream);
+        case 4128: return launch_bits_gs<4, 128>(g, bt, ksplit, stream);
+        default: return LOWBIT_ERR_UNSUPPORTED;
+    }
+}
+
+lowbit_status read_device_status(int clear) {
+    unsigned v = 0;
+    if (cudaDeviceSynchronize() != cudaSuccess) return LOWBIT_ERR_CUDA;
+    if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(v)) != cudaSuccess) return LOWBIT_ERR_CUDA;
+    if (clear && v) {
+        const unsigned zero = 0;
+        if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(zero)) != cudaSuccess) return LOWBIT_ERR_CUDA;
+    }
+    return (v & kDevErrTimeout) ? LOWBIT_ERR_TIMEOUT : LOWBIT_OK;
+}
+
+}  // namespace lowbit

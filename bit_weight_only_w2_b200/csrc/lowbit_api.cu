@@ -1,0 +1,181 @@
+// The C ABI of liblowbit.so (declared in include/lowbit.h): argument checks, the device
+// probe, and dispatch to the packing and GEMM kernels. Every check runs before any launch.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstdlib>
+#include <mutex>
+
+#include "lowbit_internal.h"
+
+#define LOWBIT_API extern "C" __attribute__((visibility("default")))
+
+namespace lowbit {
+namespace {
+
+std::mutex g_pack_mutex;   // pack / unpack share one device-side error counter
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool valid_bits(int bits) { return bits == 1 || bits == 2 || bits == 4; }
+
+lowbit_status check_pack_args(const void* a, const void* b, int64_t N, int64_t K, int bits) {
+    if (!valid_bits(bits) || N < 0 || K < 0) return LOWBIT_ERR_INVALID_ARG;
+    if (K % (32 / bits) != 0) return LOWBIT_ERR_INVALID_ARG;
+    if (N == 0 || K == 0) return LOWBIT_OK;
+    if (!a || !b) return LOWBIT_ERR_INVALID_ARG;
+    if (!aligned16(a) || !aligned16(b)) return LOWBIT_ERR_ALIGNMENT;
+    return LOWBIT_OK;
+}
+
+}  // namespace
+
+lowbit_status check_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return LOWBIT_ERR_CUDA;
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+        return LOWBIT_ERR_CUDA;
+    // The kernels are built for sm_100a only (tcgen05 / tensor memory).
+    if (major != 10 || minor != 0) return LOWBIT_ERR_UNSUPPORTED_DEVICE;
+    return LOWBIT_OK;
+}
+
+lowbit_status validate_gemm(const GemmProblem& g) {
+    if (!valid_bits(g.bits)) return LOWBIT_ERR_INVALID_ARG;
+    if (g.M < 0 || g.N < 0 || g.K <= 0 || g.group_size <= 0) return LOWBIT_ERR_INVALID_ARG;
+    if (g.K % g.group_size != 0 || g.group_size % (32 / g.bits) != 0) return LOWBIT_ERR_INVALID_ARG;
+    if ((g.bits == 4) != (g.zeros != nullptr)) return LOWBIT_ERR_INVALID_ARG;
+    if (g.M == 0 || g.N == 0) return LOWBIT_OK;
+    if (!g.X || !g.Wp || !g.scales || !g.Y) return LOWBIT_ERR_INVALID_ARG;
+    if (!aligned16(g.X) || !aligned16(g.Wp) || !aligned16(g.scales) || !aligned16(g.Y) ||
+        (g.zeros && !aligned16(g.zeros)))
+        return LOWBIT_ERR_ALIGNMENT;
+    // GPU path limits (TMA strides must be multiples of 16 bytes; supported tile configs).
+    if (g.group_size != 64 && g.group_size != 128) return LOWBIT_ERR_UNSUPPORTED;
+    if (g.bits == 1 && g.K % 128 != 0) return LOWBIT_ERR_UNSUPPORTED;
+    if (g.N % 8 != 0) return LOWBIT_ERR_UNSUPPORTED;
+    if (g.M >= (int64_t(1) << 31) || g.N >= (int64_t(1) << 31) || g.K >= (int64_t(1) << 31))
+        return LOWBIT_ERR_UNSUPPORTED;
+    return LOWBIT_OK;
+}
+
+}  // namespace lowbit
+
+using namespace lowbit;
+
+LOWBIT_API const char* lowbit_status_string(lowbit_status s) {
+    switch (s) {
+        case LOWBIT_OK: return "LOWBIT_OK";
+        case LOWBIT_ERR_INVALID_ARG: return "LOWBIT_ERR_INVALID_ARG";
+        case LOWBIT_ERR_ALIGNMENT: return "LOWBIT_ERR_ALIGNMENT";
+        case LOWBIT_ERR_UNSUPPORTED: return "LOWBIT_ERR_UNSUPPORTED";
+        case LOWBIT_ERR_UNSUPPORTED_DEVICE: return "LOWBIT_ERR_UNSUPPORTED_DEVICE";
+        case LOWBIT_ERR_BAD_CODE: return "LOWBIT_ERR_BAD_CODE";
+        case LOWBIT_ERR_TIMEOUT: return "LOWBIT_ERR_TIMEOUT";
+        case LOWBIT_ERR_CUDA: return "LOWBIT_ERR_CUDA";
+    }
+    return "LOWBIT_ERR_UNKNOWN";
+}
+
+LOWBIT_API int lowbit_version(void) { return 100; }
+
+LOWBIT_API size_t lowbit_packed_words(int64_t N, int64_t K, int bits) {
+    if (!valid_bits(bits) || N < 0 || K < 0 || K % (32 / bits) != 0) return 0;
+    return static_cast<size_t>(N) * static_cast<size_t>(K) * bits / 32;
+}
+
+LOWBIT_API lowbit_status lowbit_pack(const int8_t* codes, int64_t N, int64_t K, int bits, uint32_t* packed,
+                                     void* stream) {
+    lowbit_status st = check_pack_args(codes, packed, N, K, bits);
+    if (st != LOWBIT_OK || N == 0 || K == 0) return st;
+    if ((st = check_device()) != LOWBIT_OK) return st;
+    std::lock_guard<std::mutex> lock(g_pack_mutex);
+    unsigned long long bad = 0;
+    st = pack_launch(codes, N, K, bits, packed, static_cast<cudaStream_t>(stream), &bad);
+    if (st != LOWBIT_OK) return st;
+    return bad ? LOWBIT_ERR_BAD_CODE : LOWBIT_OK;
+}
+
+LOWBIT_API lowbit_status lowbit_unpack(const uint32_t* packed, int64_t N, int64_t K, int bits, int8_t* codes,
+                                       void* stream) {
+    lowbit_status st = check_pack_args(packed, codes, N, K, bits);
+    if (st != LOWBIT_OK || N == 0 || K == 0) return st;
+    if ((st = check_device()) != LOWBIT_OK) return st;
+    std::lock_guard<std::mutex> lock(g_pack_mutex);
+    unsigned long long bad = 0;
+    st = unpack_launch(packed, N, K, bits, codes, static_cast<cudaStream_t>(stream), &bad);
+    if (st != LOWBIT_OK) return st;
+    return bad ? LOWBIT_ERR_BAD_CODE : LOWBIT_OK;
+}
+
+static GemmProblem make_problem(int64_t M, int64_t N, int64_t K, int bits, int group_size, const void* X,
+                                const uint32_t* Wp, const void* scales, const void* zeros, void* Y) {
+    GemmProblem g;
+    g.M = M;
+    g.N = N;
+    g.K = K;
+    g.bits = bits;
+    g.group_size = group_size;
+    g.X = X;
+    g.Wp = Wp;
+    g.scales = scales;
+    g.zeros = zeros;
+    g.Y = Y;
+    return g;
+}
+
+LOWBIT_API lowbit_status lowbit_gemm(int64_t M, int64_t N, int64_t K, int bits, int group_size, const void* X,
+                                     const uint32_t* Wp, const void* scales, const void* zeros, void* Y,
+                                     void* stream) {
+    const GemmProblem g = make_problem(M, N, K, bits, group_size, X, Wp, scales, zeros, Y);
+    lowbit_status st = validate_gemm(g);
+    if (st != LOWBIT_OK || M == 0 || N == 0) return st;
+    if ((st = check_device()) != LOWBIT_OK) return st;
+    return gemm_launch(g, 0, 0, static_cast<cudaStream_t>(stream));
+}
+
+LOWBIT_API lowbit_status lowbit_gemm_ex(int64_t M, int64_t N, int64_t K, int bits, int group_size, const void* X,
+                                        const uint32_t* Wp, const void* scales, const void* zeros, void* Y,
+                                        int tile_tokens, int ksplit, void* stream) {
+    const GemmProblem g = make_problem(M, N, K, bits, group_size, X, Wp, scales, zeros, Y);
+    lowbit_status st = validate_gemm(g);
+    if (st != LOWBIT_OK || M == 0 || N == 0) return st;
+    if (tile_tokens != 0 && tile_tokens != 16 && tile_tokens != 32 && tile_tokens != 64 && tile_tokens != 128 &&
+        tile_tokens != 256)
+        return LOWBIT_ERR_UNSUPPORTED;
+    if (ksplit < 0 || ksplit > 8) return LOWBIT_ERR_UNSUPPORTED;
+    if ((st = check_device()) != LOWBIT_OK) return st;
+    return gemm_launch(g, tile_tokens, ksplit, static_cast<cudaStream_t>(stream));
+}
+
+LOWBIT_API lowbit_status lowbit_gemm_batch(const lowbit_gemm_desc* descs, int count, void* stream) {
+    if (count < 0 || (count > 0 && !descs)) return LOWBIT_ERR_INVALID_ARG;
+    for (int i = 0; i < count; ++i) {
+        const lowbit_gemm_desc& d = descs[i];
+        const lowbit_status st = validate_gemm(
+            make_problem(d.M, d.N, d.K, d.bits, d.group_size, d.X, d.Wp, d.scales, d.zeros, d.Y));
+        if (st != LOWBIT_OK) return st;
+    }
+    if (count == 0) return LOWBIT_OK;
+    lowbit_status st = check_device();
+    if (st != LOWBIT_OK) return st;
+    for (int i = 0; i < count; ++i) {
+        const lowbit_gemm_desc& d = descs[i];
+        if (d.M == 0 || d.N == 0) continue;
+        st = gemm_launch(make_problem(d.M, d.N, d.K, d.bits, d.group_size, d.X, d.Wp, d.scales, d.zeros, d.Y),
+                         0, 0, static_cast<cudaStream_t>(stream));
+        if (st != LOWBIT_OK) return st;
+    }
+    return LOWBIT_OK;
+}
+
+LOWBIT_API lowbit_status lowbit_device_status(int clear) { return read_device_status(clear); }
+
+LOWBIT_API lowbit_status lowbit_selftest_bounded_wait(long long limit_cycles, void* stream) {
+    if (limit_cycles <= 0) return LOWBIT_ERR_INVALID_ARG;
+    const lowbit_status st = check_device();
+    if (st != LOWBIT_OK) return st;
+    return selftest_bounded_wait(limit_cycles, static_cast<cudaStream_t>(stream));
+}

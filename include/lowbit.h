@@ -1,0 +1,137 @@
+/*
+ * lowbit.h -- C ABI of liblowbit.so: weight-only low-bit GEMM for NVIDIA B200 (sm_100a).
+ *
+ *   Y[M][N] = X[M][K] * W^T,   W[N][K] decoded from packed low-bit codes and fp16 group scales.
+ *
+ * This is the matrix multiply behind the Q/K/V, output and MLP linears of the Bonsai Image
+ * (FLUX.2-Klein-4B) transformer, whose weights are binary 1-bit with one FP16 scale per group
+ * of 128 (bonsai-image-binary-4B-gemlite-1bit model card, "Binary Weight Representation:
+ * 1-bit g128") or ternary 2-bit (mlx-vlm Bonsai article, model overview), and of the 4-bit
+ * grouped text-encoder linears, group 64 (same article, component architecture).
+ *
+ * Formats (bits):
+ *   1  binary   w = s * b,        b in {-1,+1}         code values -1 / +1
+ *   2  ternary  w = s * t,        t in {-1, 0,+1}      code values -1 / 0 / +1
+ *   4  uint4    w = (q - z) * s,  q in 0..15           code values 0..15, z = per-group zero
+ * s and z are fp16, one per group of `group_size` consecutive K elements of one output row.
+ *
+ * Packed code layout (uint32 words, packed along K; produced by lowbit_pack):
+ *   cpw = 32 / bits codes per word; row n of W owns words [n*K/cpw, (n+1)*K/cpw).
+ *   The code of column k is in word k / cpw at offset i = k % cpw, in bits
+ *   [pos, pos + bits) with pos = (i % 2) * 16 + (i / 2) * bits: even offsets fill the low
+ *   16 bits and odd offsets the high 16 bits, each half LSB-first. Stored fields:
+ *   binary +1 -> 1, -1 -> 0; ternary t -> t + 1 (3 is invalid); uint4 q -> q.
+ *   (The pages pack codes along K into uint32 words -- Bonsai-Image-Demo PR #20, GemLite
+ *   int2 layout note; image-studio backend.md, checkpoint layout -- but leave the bit order
+ *   open. This order puts the two codes of a K pair in the two bf16 halves of one 32-bit
+ *   register, so a decoder builds bf16x2 operands with one mask per pair.)
+ *
+ * Scale / zero layout: fp16, group-major [K/group_size][N]: s(n, k) = scales[(k/g)*N + n].
+ * X: bf16 row-major [M][K]. Y: bf16 row-major [M][N]. Accumulation is fp32.
+ *
+ * Ownership: the caller owns every buffer (device memory unless stated). The library keeps
+ * no allocation; it holds one small status word per device in static device memory.
+ * Streams are CUDA stream handles (cudaStream_t) passed as void*; NULL = legacy stream.
+ * Errors: argument / shape errors return before any launch and change nothing.
+ */
+#ifndef LOWBIT_H_
+#define LOWBIT_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum lowbit_status {
+    LOWBIT_OK = 0,
+    LOWBIT_ERR_INVALID_ARG = 1,        /* NULL pointer, bad bits / group size, bad shape        */
+    LOWBIT_ERR_ALIGNMENT = 2,          /* a pointer is not 16-byte aligned                      */
+    LOWBIT_ERR_UNSUPPORTED = 3,        /* valid problem the GPU path does not take (see below)  */
+    LOWBIT_ERR_UNSUPPORTED_DEVICE = 4, /* current device is not sm_100 (B200 class)             */
+    LOWBIT_ERR_BAD_CODE = 5,           /* pack: a code outside its format; unpack: field 3       */
+    LOWBIT_ERR_TIMEOUT = 6,            /* a bounded wait inside a kernel gave up (device status) */
+    LOWBIT_ERR_CUDA = 7                /* a CUDA runtime / driver call failed                    */
+} lowbit_status;
+
+/* Human-readable name of a status. Never NULL. */
+const char* lowbit_status_string(lowbit_status s);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int lowbit_version(void);
+
+/* Number of uint32 words of the packed codes of an [N][K] weight: N * K * bits / 32.
+ * Returns 0 for invalid arguments (bits not 1/2/4, K not a multiple of 32/bits, N or K < 0). */
+size_t lowbit_packed_words(int64_t N, int64_t K, int bits);
+
+/* Pack int8 codes [N][K] (device, row-major) into `packed` [N][K*bits/32] uint32 (device),
+ * in the layout above. Validates every code: on any invalid code returns
+ * LOWBIT_ERR_BAD_CODE (the packed buffer is then unspecified). Synchronous: waits for the
+ * work on `stream`. Requires K % (32/bits) == 0; codes 16-byte aligned when K > 0.
+ * Calls are serialised inside the library (they share one device-side error counter). */
+lowbit_status lowbit_pack(const int8_t* codes, int64_t N, int64_t K, int bits, uint32_t* packed,
+                          void* stream);
+
+/* Inverse of lowbit_pack: packed [N][K*bits/32] -> int8 codes [N][K] (device). Returns
+ * LOWBIT_ERR_BAD_CODE if a ternary field holds 3 (written as 0). Synchronous, serialised. */
+lowbit_status lowbit_unpack(const uint32_t* packed, int64_t N, int64_t K, int bits, int8_t* codes,
+                            void* stream);
+
+/* Y = X * W^T on `stream` (asynchronous; never synchronises).
+ *   X       [M][K]            bf16, device, 16-byte aligned
+ *   Wp      [N][K*bits/32]    uint32 packed codes, device, 16-byte aligned
+ *   scales  [K/group_size][N] fp16, device, 16-byte aligned
+ *   zeros   [K/group_size][N] fp16 for bits == 4, NULL otherwise
+ *   Y       [M][N]            bf16, device, 16-byte aligned; must not overlap the inputs
+ * GPU path preconditions (else LOWBIT_ERR_UNSUPPORTED): group_size 64 or 128,
+ * K % group_size == 0, K % 128 == 0 when bits == 1, N % 8 == 0, M, N, K < 2^31.
+ * M == 0 or N == 0 is a no-op. Kernel-side bounded waits that give up set the device
+ * status word (see lowbit_device_status) instead of trapping. */
+lowbit_status lowbit_gemm(int64_t M, int64_t N, int64_t K, int bits, int group_size, const void* X,
+                          const uint32_t* Wp, const void* scales, const void* zeros, void* Y,
+                          void* stream);
+
+/* lowbit_gemm with the kernel configuration fixed instead of chosen from the shape, for
+ * tuning and tests: `tile_tokens` = tokens per CTA tile (16, 32, 64, 128 or 256; 0 = automatic),
+ * `ksplit` = number of K slices summed across a thread-block cluster (1..8; 0 = automatic,
+ * 1 = no split). Other arguments and all checks are those of lowbit_gemm; an unsupported
+ * tile_tokens returns LOWBIT_ERR_UNSUPPORTED. */
+lowbit_status lowbit_gemm_ex(int64_t M, int64_t N, int64_t K, int bits, int group_size, const void* X,
+                             const uint32_t* Wp, const void* scales, const void* zeros, void* Y,
+                             int tile_tokens, int ksplit, void* stream);
+
+/* One linear of a chain, with the meaning and layout of lowbit_gemm's arguments. */
+typedef struct lowbit_gemm_desc {
+    int64_t M, N, K;
+    int bits, group_size;
+    const void* X;
+    const uint32_t* Wp;
+    const void* scales;
+    const void* zeros;
+    void* Y;
+} lowbit_gemm_desc;
+
+/* Run `count` GEMMs (host array of descriptors) in order on `stream`, as if lowbit_gemm were
+ * called for each in turn: a descriptor may read an earlier one's Y. All descriptors are
+ * validated first; on any invalid one nothing is launched and its error is returned.
+ * Consecutive launches overlap their prologues with the previous kernel's tail
+ * (programmatic dependent launch); results are the same as separate calls. */
+lowbit_status lowbit_gemm_batch(const lowbit_gemm_desc* descs, int count, void* stream);
+
+/* Read the current device's sticky status word, written by kernels whose bounded waits gave
+ * up (LOWBIT_ERR_TIMEOUT), and clear it when `clear` != 0. Synchronises the device. */
+lowbit_status lowbit_device_status(int clear);
+
+/* Diagnostic for the kernels' failure detection: launches one CTA that waits on a
+ * shared-memory barrier nothing ever completes, using the same bounded wait as the GEMM kernel
+ * but giving up after `limit_cycles` SM clocks (> 0). The wait then records LOWBIT_ERR_TIMEOUT in
+ * the device status word and the kernel returns normally, so the context stays usable; read it
+ * with lowbit_device_status. Asynchronous. */
+lowbit_status lowbit_selftest_bounded_wait(long long limit_cycles, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LOWBIT_H_ */

@@ -1,0 +1,105 @@
+"""The C ABI without a GPU: the library loads, exports every function its header declares,
+and rejects invalid arguments before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import bit_weight_only_w2_b200 as lb
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADERS = [os.path.join(ROOT, "include", f) for f in os.listdir(os.path.join(ROOT, "include")) if f.endswith(".h")]
+
+
+def declared_functions():
+    names = set()
+    for h in HEADERS:
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"^[A-Za-z_][\w \*]*?\b(lowbit_\w+)\s*\(", text, flags=re.M):
+            names.add(m.group(1))
+    return sorted(names)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return lb.load()
+
+
+def test_header_declares_entry_points():
+    names = declared_functions()
+    for required in ("lowbit_pack", "lowbit_unpack", "lowbit_gemm", "lowbit_gemm_batch", "lowbit_gemm_ex",
+                     "lowbit_packed_words", "lowbit_device_status", "lowbit_status_string"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} declared in include/ but not exported"
+
+
+def test_host_functions(lib):
+    assert lib.lowbit_version() >= 100
+    assert lib.lowbit_status_string(0) == b"LOWBIT_OK"
+    assert lib.lowbit_status_string(5) == b"LOWBIT_ERR_BAD_CODE"
+    assert lib.lowbit_status_string(99) == b"LOWBIT_ERR_UNKNOWN"
+    assert lib.lowbit_packed_words(9216, 3072, 2) == 9216 * 3072 // 16
+    assert lib.lowbit_packed_words(4, 64, 1) == 8
+    assert lib.lowbit_packed_words(4, 48, 1) == 0      # K not a multiple of 32
+    assert lib.lowbit_packed_words(4, 64, 3) == 0      # bits
+    assert lib.lowbit_packed_words(-1, 64, 2) == 0
+
+
+A = 1 << 20  # a fake 16-byte-aligned address: never dereferenced, checks fail first
+
+
+@pytest.mark.parametrize("args,expect", [
+    (dict(bits=3), 1),
+    (dict(group_size=0), 1),
+    (dict(K=100), 1),                       # K not a multiple of the group size
+    (dict(zeros=A), 1),                     # zeros with bits != 4
+    (dict(bits=4), 1),                      # bits 4 without zeros
+    (dict(X=0), 1),                         # NULL input
+    (dict(X=A + 2), 2),                     # misaligned
+    (dict(Y=A + 8), 2),
+    (dict(group_size=32, K=256), 3),        # GPU path takes groups of 64 / 128 only
+    (dict(N=100), 3),                       # N % 8
+    (dict(bits=1, K=192, group_size=64), 3),  # binary needs K % 128
+    (dict(M=-1), 1),
+])
+def test_gemm_rejects_before_launch(lib, args, expect):
+    a = dict(M=16, N=128, K=256, bits=2, group_size=128, X=A, Wp=A, scales=A, zeros=0, Y=A)
+    a.update(args)
+    st = lib.lowbit_gemm(a["M"], a["N"], a["K"], a["bits"], a["group_size"], a["X"], a["Wp"], a["scales"],
+                         a["zeros"] or None, a["Y"], None)
+    assert st == expect, lb.STATUS.get(st)
+
+
+def test_gemm_ex_rejects_bad_tile(lib):
+    st = lib.lowbit_gemm_ex(16, 128, 256, 2, 128, A, A, A, None, A, 48, 0, None)
+    assert st == 3
+    st = lib.lowbit_gemm_ex(16, 128, 256, 2, 128, A, A, A, None, A, 16, 9, None)
+    assert st == 3
+
+
+def test_batch_validates_all_first(lib):
+    good = lb.GemmDesc(16, 128, 256, 2, 128, A, A, A, None, A)
+    bad = lb.GemmDesc(16, 128, 256, 3, 128, A, A, A, None, A)
+    arr = (lb.GemmDesc * 2)(good, bad)
+    assert lib.lowbit_gemm_batch(arr, 2, None) == 1
+    assert lib.lowbit_gemm_batch(None, -1, None) == 1
+    assert lib.lowbit_gemm_batch(None, 0, None) == 0
+
+
+def test_empty_problems_are_noops(lib):
+    assert lib.lowbit_gemm(0, 128, 256, 2, 128, A, A, A, None, A, None) == 0
+    assert lib.lowbit_gemm(16, 0, 256, 2, 128, A, A, A, None, A, None) == 0
+    assert lib.lowbit_pack(None, 0, 64, 2, None, None) == 0
+
+
+def test_pack_rejects_before_launch(lib):
+    assert lib.lowbit_pack(A, 4, 48, 1, A, None) == 1       # K % 32
+    assert lib.lowbit_pack(A, 4, 64, 3, A, None) == 1
+    assert lib.lowbit_pack(A + 1, 4, 64, 2, A, None) == 2
+    assert lib.lowbit_unpack(None, 4, 64, 2, A, None) == 1
