@@ -23,6 +23,7 @@ LIB_PATH = os.path.join(_HERE, "liblowbit.so")
 STATUS = {
     0: "LOWBIT_OK", 1: "LOWBIT_ERR_INVALID_ARG", 2: "LOWBIT_ERR_ALIGNMENT", 3: "LOWBIT_ERR_UNSUPPORTED",
     4: "LOWBIT_ERR_UNSUPPORTED_DEVICE", 5: "LOWBIT_ERR_BAD_CODE", 6: "LOWBIT_ERR_TIMEOUT", 7: "LOWBIT_ERR_CUDA",
+    8: "LOWBIT_ERR_WORKSPACE",
 }
 
 
@@ -60,11 +61,14 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.lowbit_pack.restype = i32
     lib.lowbit_unpack.argtypes = [p, i64, i64, i32, p, p]
     lib.lowbit_unpack.restype = i32
-    lib.lowbit_gemm.argtypes = [i64, i64, i64, i32, i32, p, p, p, p, p, p]
+    sz = ctypes.c_size_t
+    lib.lowbit_gemm_workspace_size.argtypes = [i64, i64]
+    lib.lowbit_gemm_workspace_size.restype = sz
+    lib.lowbit_gemm.argtypes = [i64, i64, i64, i32, i32, p, p, p, p, p, p, sz, p]
     lib.lowbit_gemm.restype = i32
-    lib.lowbit_gemm_ex.argtypes = [i64, i64, i64, i32, i32, p, p, p, p, p, i32, i32, p]
+    lib.lowbit_gemm_ex.argtypes = [i64, i64, i64, i32, i32, p, p, p, p, p, p, sz, i32, i32, p]
     lib.lowbit_gemm_ex.restype = i32
-    lib.lowbit_gemm_batch.argtypes = [ctypes.POINTER(GemmDesc), i32, p]
+    lib.lowbit_gemm_batch.argtypes = [ctypes.POINTER(GemmDesc), i32, p, sz, p]
     lib.lowbit_gemm_batch.restype = i32
     lib.lowbit_device_status.argtypes = [i32]
     lib.lowbit_device_status.restype = i32
@@ -120,9 +124,29 @@ def unpack(packed: torch.Tensor, N: int, K: int, bits: int) -> torch.Tensor:
     return out
 
 
+def workspace_size(M: int, K: int) -> int:
+    return int(load().lowbit_gemm_workspace_size(M, K))
+
+
+_workspaces = {}
+
+
+def workspace(device: torch.device, nbytes: int) -> torch.Tensor:
+    """A cached per-device workspace buffer of at least `nbytes` (grown on demand). Work that
+    uses it is ordered on the current stream; callers running GEMMs on several streams at once
+    should pass their own buffers."""
+    dev = torch.device(device)
+    key = dev.index if dev.index is not None else torch.cuda.current_device()
+    buf = _workspaces.get(key)
+    if buf is None or buf.numel() < nbytes:
+        buf = torch.empty(max(nbytes, 1 << 20), dtype=torch.uint8, device=torch.device("cuda", key))
+        _workspaces[key] = buf
+    return buf
+
+
 def gemm(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, zeros: Optional[torch.Tensor],
          bits: int, group_size: int, out: Optional[torch.Tensor] = None, tile_tokens: int = 0,
-         ksplit: int = 0) -> torch.Tensor:
+         ksplit: int = 0, ws: Optional[torch.Tensor] = None) -> torch.Tensor:
     """Y[M][N] = X[M][K] * W^T with W decoded from `packed`, `scales` (and `zeros`)."""
     _need(x, torch.bfloat16, "x")
     _need(packed, torch.int32, "packed")
@@ -137,12 +161,15 @@ def gemm(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, zeros: Opt
         _need(out, torch.bfloat16, "out")
     with torch.cuda.device(x.device):
         lib = load()
+        need = workspace_size(M, K)
+        if ws is None:
+            ws = workspace(x.device, need)
         if tile_tokens or ksplit:
             st = lib.lowbit_gemm_ex(M, N, K, bits, group_size, _ptr(x), _ptr(packed), _ptr(scales), _ptr(zeros),
-                                    _ptr(out), tile_tokens, ksplit, _stream(x))
+                                    _ptr(out), _ptr(ws), ws.numel(), tile_tokens, ksplit, _stream(x))
         else:
             st = lib.lowbit_gemm(M, N, K, bits, group_size, _ptr(x), _ptr(packed), _ptr(scales), _ptr(zeros),
-                                 _ptr(out), _stream(x))
+                                 _ptr(out), _ptr(ws), ws.numel(), _stream(x))
         _check(st, "lowbit_gemm")
     return out
 
@@ -153,11 +180,16 @@ def make_desc(x, packed, scales, zeros, y, bits: int, group_size: int) -> GemmDe
     return GemmDesc(M, N, K, bits, group_size, _ptr(x), _ptr(packed), _ptr(scales), _ptr(zeros), _ptr(y))
 
 
-def gemm_batch(descs: Sequence[GemmDesc], device: Optional[torch.device] = None) -> None:
+def gemm_batch(descs: Sequence[GemmDesc], device: Optional[torch.device] = None,
+               ws: Optional[torch.Tensor] = None) -> None:
     """Run the descriptors in order on the current stream (see lowbit_gemm_batch)."""
     arr = (GemmDesc * len(descs))(*descs)
-    with torch.cuda.device(device if device is not None else torch.cuda.current_device()):
-        _check(load().lowbit_gemm_batch(arr, len(descs), _stream()), "lowbit_gemm_batch")
+    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    with torch.cuda.device(dev):
+        if ws is None:
+            need = max((workspace_size(d.M, d.K) for d in descs), default=0)
+            ws = workspace(dev, need)
+        _check(load().lowbit_gemm_batch(arr, len(descs), _ptr(ws), ws.numel(), _stream()), "lowbit_gemm_batch")
 
 
 def device_status(clear: bool = True) -> int:

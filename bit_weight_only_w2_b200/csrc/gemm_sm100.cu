@@ -8,19 +8,28 @@
 // architecture). After decoding it is a dense contraction, so it runs on the tcgen05 tensor
 // cores.
 //
+// Precision: the tensor cores run in fp16 with fp32 accumulation. A pre-pass converts X from
+// bf16 to fp16 (exact: every bf16 value in fp16's normal range is an fp16 value), with a
+// per-row power-of-two scale so that rows whose magnitude exceeds fp16's range still convert
+// exactly (the epilogue multiplies that row back). In fp16 a binary or ternary weight t * s is
+// exactly +-s or 0 for the fp16 scale s, and a uint4 weight (q - z) * s is rounded once to fp16
+// (2^-11 relative); rounding s to bf16 instead would cost up to 2^-8 per group, enough to
+// break a 1e-2 tolerance in the tails.
+//
 // Kernel design ("swap AB", weights as the MMA's A operand):
 //   * One CTA tile = 128 weight rows (MMA M) x BT tokens (MMA N), K in stages of 128.
 //   * Warp 0 (one lane) is the TMA producer: per stage it loads two 64-wide, 128B-swizzled
-//     boxes of X (the MMA's B operand, K-major), the packed code box of the 128 rows and their
+//     boxes of the fp16 copy of X (the MMA's B operand, K-major), the packed code box of the 128 rows and their
 //     group scales (and zeros) into a shared-memory ring.
 //   * The dequant warps each own 32 weight rows (one per lane, matching the tensor-memory lane
 //     quarter the warp may access): they read the row's packed words from shared memory,
-//     decode codes x scale to bf16 pairs with a few integer / bf16x2 instructions per pair,
+//     decode codes x scale to fp16 pairs with a few integer / fp16x2 instructions per pair,
 //     and store them straight into a tensor-memory ring with tcgen05.st. The decoded weights
 //     never touch shared memory, which leaves its bandwidth to TMA and the MMA's B reads.
 //   * Warp 1 (one lane) issues tcgen05.mma (kind::f16, A from tensor memory, B from shared
 //     memory, fp32 accumulators in tensor memory) and frees ring slots with tcgen05.commit.
-//   * Four epilogue warps read the accumulators with tcgen05.ld, round to bf16 and store Y.
+//   * Four epilogue warps read the accumulators with tcgen05.ld, apply the row's power-of-two
+//     scale, round to bf16 and store Y.
 //     With two accumulator buffers the epilogue of one tile overlaps the next tile's MMAs.
 //   * Without split-K the grid is persistent (tiles strided over the CTAs). With split-K
 //     (small M, few tiles) the K range is divided over the CTAs of a thread-block cluster and
@@ -70,7 +79,7 @@ struct Cfg {
 
     static constexpr int kWordsPerRow = kBlockK * BITS / 32;        // 4 / 8 / 16
     static constexpr int kWRowBytes = kWordsPerRow * 4;             // 16 / 32 / 64
-    static constexpr int kXHalfBytes = BT * 128;                    // 64 bf16 per row
+    static constexpr int kXHalfBytes = BT * 128;                    // 64 fp16 per row
     static constexpr int kXBytes = 2 * kXHalfBytes;
     static constexpr int kWBytes = kBlockN * kWRowBytes;
     static constexpr int kGroupsPerStage = kBlockK / GS;            // 1 or 2
@@ -96,7 +105,7 @@ struct Cfg {
     static_assert(kSmemBytes <= kSmemLimit, "shared memory");
     // split-K partial tile (fp32 [BT][128]) reuses the stage ring
     static_assert(BT * kBlockN * 4 <= kStages * kStageBytes, "split-K partial buffer");
-    static constexpr uint32_t kIdesc = idesc_bf16_f32(kBlockN, BT);
+    static constexpr uint32_t kIdesc = idesc_f16_f32(kBlockN, BT);
 };
 
 struct KernelParams {
@@ -106,15 +115,16 @@ struct KernelParams {
     int m_tiles, n_tiles, num_tiles;
     int ksplit;          // cluster size along z (1 = persistent, no split)
     __nv_bfloat16* Y;
+    const float* rowmul; // per-row power-of-two factor written by the X conversion pass
 };
 
 // ---------------------------------------------------------------------------------------------
-// Decoders: one 64-wide K half of one weight row -> 32 bf16x2 values (even k low, odd k high).
+// Decoders: one 64-wide K half of one weight row -> 32 fp16x2 values (even k low, odd k high).
 // ---------------------------------------------------------------------------------------------
 
 // Binary: bit 1 -> +s, 0 -> -s. Pair c of a word is (bit c, bit 16 + c); shifting the word
-// left by 15 - c puts them on the two bf16 sign bits, and one LOP3 flips the sign of s where
-// the bit is 0. Exact: the result is +-bf16(s).
+// left by 15 - c puts them on the two fp16 sign bits, and one LOP3 flips the sign of s where
+// the bit is 0. Exact.
 __device__ __forceinline__ void decode_half_b1(uint32_t w0, uint32_t w1, uint32_t s2, uint32_t (&out)[32]) {
 #pragma unroll
     for (int c = 0; c < 16; ++c) out[c] = xor_andnot(s2, w0 << (15 - c), 0x80008000u);
@@ -122,41 +132,40 @@ __device__ __forceinline__ void decode_half_b1(uint32_t w0, uint32_t w1, uint32_
     for (int c = 0; c < 16; ++c) out[16 + c] = xor_andnot(s2, w1 << (15 - c), 0x80008000u);
 }
 
-// Ternary: field f = t + 1 in {0,1,2}. OR-ing the two fields of a pair into the mantissas of
-// bf16 128.0 gives (128 + f * 4^j) exactly (j = field position inside the mantissa); one
-// bf16x2 FMA subtracts (128 + 4^j), leaving t * 4^j exactly, and a second multiplies by
-// s * 4^-j, giving t * s exactly (t in {-1,0,1}). s4[j] holds bf16x2(s * 4^-j).
-__device__ __forceinline__ void decode_word_b2(uint32_t v, const uint32_t (&s4)[3], uint32_t* out) {
-    constexpr uint32_t kMagic = 0x43004300u;                           // bf16x2(128, 128)
-    constexpr uint32_t kOne = 0x3F803F80u;                             // bf16x2(1, 1)
-    constexpr uint32_t kNegBase[3] = {0xC301C301u, 0xC304C304u, 0xC310C310u};  // -(128 + 4^j)
-    constexpr uint32_t kNegZero = 0x80008000u;
+// Ternary: field f = t + 1 in {0,1,2}. OR-ing the two fields of a pair, left at bit 2j of each
+// half, into the mantissas of fp16 1024.0 gives e = 1024 + f * 4^j exactly (j <= 4 keeps the
+// field inside the 10-bit mantissa). One fp16x2 FMA computes e * 4^-j - (1024 * 4^-j + 1) =
+// f - 1 = t exactly (the exact result is representable, so nothing rounds) and a multiply by
+// s gives t * s exactly. Pairs 0..4 are decoded in place, pairs 5..7 after one shift by 10.
+__device__ __forceinline__ void decode_word_b2(uint32_t v, uint32_t s2, uint32_t* out) {
+    constexpr uint32_t kMagic = 0x64006400u;                                           // 1024.0
+    constexpr uint32_t kMul[5] = {0x3C003C00u, 0x34003400u, 0x2C002C00u, 0x24002400u, 0x1C001C00u};  // 4^-j
+    constexpr uint32_t kAdd[5] = {0xE401E401u, 0xDC04DC04u, 0xD410D410u, 0xCC40CC40u, 0xC500C500u};  // -(1024*4^-j+1)
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
-        const int shift = (c / 3) * 6;
-        const int j = c % 3;
+        const int shift = (c < 5) ? 0 : 10;
+        const int j = (c < 5) ? c : c - 5;
         const uint32_t e = and_or(v >> shift, 0x00030003u << (2 * j), kMagic);
-        const uint32_t t = bf16x2_fma(e, kOne, kNegBase[j]);
-        out[c] = bf16x2_fma(t, s4[j], kNegZero);
+        const uint32_t t = f16x2_fma(e, kMul[j], kAdd[j]);
+        out[c] = f16x2_mul(t, s2);
     }
 }
 
-// uint4: OR-ing a nibble into bits 16..19 of fp32 128.0 gives 128 + q exactly; one FMA with
-// s and c = -(128 + z) * s gives (q - z) * s to fp32 rounding, then a pair is rounded to bf16.
-__device__ __forceinline__ void decode_word_b4(uint32_t v, float s, float cz, uint32_t* out) {
-    constexpr uint32_t kMagic = 0x43000000u;   // fp32 128.0
+// uint4: the nibbles of a pair, left at bit 4j of each half (j <= 1), OR-ed into fp16 1024.0
+// give 1024 + q * 16^j exactly; one FMA recovers q exactly and a second computes
+// q * s + (-z * s), rounded once to fp16. c2 = fp16x2(-z * s) of the group.
+__device__ __forceinline__ void decode_word_b4(uint32_t v, uint32_t s2, uint32_t c2, uint32_t* out) {
+    constexpr uint32_t kMagic = 0x64006400u;
+    constexpr uint32_t kMul[2] = {0x3C003C00u, 0x2C002C00u};   // 1, 1/16
+    constexpr uint32_t kAdd[2] = {0xE400E400u, 0xD400D400u};   // -1024, -64
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
-        const uint32_t lo = and_or(v << (16 - 4 * c), 0x000F0000u, kMagic);
-        const uint32_t hi = and_or(v >> (4 * c), 0x000F0000u, kMagic);
-        out[c] = pack_bf16x2(fmaf(__uint_as_float(lo), s, cz), fmaf(__uint_as_float(hi), s, cz));
+        const int shift = (c < 2) ? 0 : 8;
+        const int j = c & 1;
+        const uint32_t e = and_or(v >> shift, 0x000F000Fu << (4 * j), kMagic);
+        const uint32_t q = f16x2_fma(e, kMul[j], kAdd[j]);
+        out[c] = f16x2_fma(q, s2, c2);
     }
-}
-
-__device__ __forceinline__ uint32_t bf16x2_splat(float f) {
-    const __nv_bfloat16 b = __float2bfloat16_rn(f);
-    const uint32_t u = static_cast<uint32_t>(__bfloat16_as_ushort(b));
-    return u | (u << 16);
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -283,7 +292,7 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT>::kThreads, Cfg<BITS, GS, BT>
                         const uint32_t a_tmem = tmem_base + C::kACol0 + a * 64 + kk * 8;
                         const uint64_t bdesc =
                             smem_desc_k_sw128(xs + (kk >> 2) * C::kXHalfBytes + (kk & 3) * 32);
-                        mma_bf16_ts(d_tmem, a_tmem, bdesc, C::kIdesc, (kb > kb_begin || kk > 0) ? 1u : 0u);
+                        mma_f16_ts(d_tmem, a_tmem, bdesc, C::kIdesc, (kb > kb_begin || kk > 0) ? 1u : 0u);
                     }
                     issued = true;
                     mma_commit(&empty[s]);
@@ -340,18 +349,21 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT>::kThreads, Cfg<BITS, GS, BT>
                         }
                     }
                 }
-                float sc[kHalvesPerPart], zc[kHalvesPerPart];
+                uint32_t s2[kHalvesPerPart], c2[kHalvesPerPart];
 #pragma unroll
                 for (int hh = 0; hh < kHalvesPerPart; ++hh) {
                     const int h = part * kHalvesPerPart + hh;
                     const int gi = (GS == 64) ? h : 0;
-                    const __half* srow = reinterpret_cast<const __half*>(st + C::kSOff) + gi * kBlockN;
-                    sc[hh] = __half2float(srow[row]);
+                    const uint16_t* srow = reinterpret_cast<const uint16_t*>(st + C::kSOff) + gi * kBlockN;
+                    const uint32_t sb = srow[row];
+                    s2[hh] = sb | (sb << 16);
                     if (BITS == 4) {
                         const __half* zrow = reinterpret_cast<const __half*>(st + C::kZOff) + gi * kBlockN;
-                        zc[hh] = __half2float(zrow[row]);
+                        const float cz = -__half2float(zrow[row]) * __half2float(__ushort_as_half(static_cast<unsigned short>(sb)));
+                        const uint32_t cb = __half_as_ushort(__float2half_rn(cz));
+                        c2[hh] = cb | (cb << 16);
                     } else {
-                        zc[hh] = 0.f;
+                        c2[hh] = 0;
                     }
                 }
                 __syncwarp();
@@ -367,16 +379,13 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT>::kThreads, Cfg<BITS, GS, BT>
                     const int h = part * kHalvesPerPart + hh;
                     uint32_t out[32];
                     if (BITS == 1) {
-                        decode_half_b1(words[hh][0], words[hh][1], bf16x2_splat(sc[hh]), out);
+                        decode_half_b1(words[hh][0], words[hh][1], s2[hh], out);
                     } else if (BITS == 2) {
-                        const uint32_t s4[3] = {bf16x2_splat(sc[hh]), bf16x2_splat(sc[hh] * 0.25f),
-                                                bf16x2_splat(sc[hh] * 0.0625f)};
 #pragma unroll
-                        for (int w = 0; w < 4; ++w) decode_word_b2(words[hh][w], s4, out + 8 * w);
+                        for (int w = 0; w < 4; ++w) decode_word_b2(words[hh][w], s2[hh], out + 8 * w);
                     } else {
-                        const float cz = -(128.0f + zc[hh]) * sc[hh];
 #pragma unroll
-                        for (int w = 0; w < 8; ++w) decode_word_b4(words[hh][w], sc[hh], cz, out + 4 * w);
+                        for (int w = 0; w < 8; ++w) decode_word_b4(words[hh][w], s2[hh], c2[hh], out + 4 * w);
                     }
                     tmem_st32(lane_base + C::kACol0 + a * 64 + h * 32, out);
                 }
@@ -409,13 +418,15 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT>::kThreads, Cfg<BITS, GS, BT>
                 }
                 tmem_wait_ld();
                 if (!split) {
-                    if (n < p.N) {
+                    // lane j holds the power-of-two factor of token m0 + c0 + j
+                    const int mj = m0 + c0 + lane;
+                    const float mul_j = (lane < kChunk && mj < p.M) ? p.rowmul[mj] : 1.0f;
 #pragma unroll
-                        for (int j = 0; j < kChunk; ++j) {
-                            const int m = m0 + c0 + j;
-                            if (m < p.M)
-                                p.Y[static_cast<size_t>(m) * p.N + n] = __float2bfloat16_rn(__uint_as_float(v[j]));
-                        }
+                    for (int j = 0; j < kChunk; ++j) {
+                        const int m = m0 + c0 + j;
+                        const float mul = __shfl_sync(0xffffffffu, mul_j, j);
+                        if (n < p.N && m < p.M)
+                            p.Y[static_cast<size_t>(m) * p.N + n] = __float2bfloat16_rn(__uint_as_float(v[j]) * mul);
                     }
                 } else {
                     float* part = reinterpret_cast<float*>(smem);
@@ -447,7 +458,7 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT>::kThreads, Cfg<BITS, GS, BT>
                     const uint32_t off = static_cast<uint32_t>((c * kBlockN + row) * 4);
                     float acc = 0.f;
                     for (int q = 0; q < p.ksplit; ++q) acc += ld_shared_cluster_f32(map_shared_rank(part0 + off, q));
-                    p.Y[static_cast<size_t>(m) * p.N + n] = __float2bfloat16_rn(acc);
+                    p.Y[static_cast<size_t>(m) * p.N + n] = __float2bfloat16_rn(acc * p.rowmul[m]);
                 }
             }
         }
@@ -460,6 +471,59 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT>::kThreads, Cfg<BITS, GS, BT>
         tc_fence_after();
         tmem_dealloc(tmem_base, C::kTmemCols);
     }
+}
+
+// ---------------------------------------------------------------------------------------------
+// X conversion pass: bf16 [M][K] -> fp16 [M][K] with a power-of-two factor per row.
+// ---------------------------------------------------------------------------------------------
+// One CTA per row: finds the largest |x| of the row (from the bf16 bits), picks e so that the
+// row's largest value scaled by 2^-e lies in [2^15, 2^16) -- inside fp16's range, with every value
+// within 2^29 of it still an fp16 normal -- writes the row times 2^-e as fp16 (exact) and
+// rowmul[row] = 2^e, which the GEMM epilogue multiplies back (exact). Rows that are all zero,
+// or hold an infinity or NaN, keep e = 0 (non-finite values convert as they are).
+__device__ __forceinline__ uint32_t absmax_bf16x8(const uint4& v, uint32_t m) {
+    m = max(m, max(v.x & 0x7FFFu, (v.x >> 16) & 0x7FFFu));
+    m = max(m, max(v.y & 0x7FFFu, (v.y >> 16) & 0x7FFFu));
+    m = max(m, max(v.z & 0x7FFFu, (v.z >> 16) & 0x7FFFu));
+    m = max(m, max(v.w & 0x7FFFu, (v.w >> 16) & 0x7FFFu));
+    return m;
+}
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w, float scale) {
+    return pack_f16x2(__uint_as_float(w << 16) * scale, __uint_as_float(w & 0xFFFF0000u) * scale);
+}
+
+constexpr int kConvThreads = 256;
+
+__global__ void __launch_bounds__(kConvThreads) convert_x_kernel(const uint4* __restrict__ X, int K8,
+                                                                 uint4* __restrict__ Xh, float* __restrict__ rowmul) {
+    grid_dependency_wait();
+    grid_launch_dependents();
+    const int row = blockIdx.x;
+    const uint4* src = X + static_cast<size_t>(row) * K8;
+    uint4* dst = Xh + static_cast<size_t>(row) * K8;
+    uint32_t mx = 0;
+    for (int i = threadIdx.x; i < K8; i += kConvThreads) mx = absmax_bf16x8(src[i], mx);
+    mx = __reduce_max_sync(0xffffffffu, mx);
+    __shared__ uint32_t warp_max[kConvThreads / 32];
+    if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = mx;
+    __syncthreads();
+    mx = 0;
+#pragma unroll
+    for (int w = 0; w < kConvThreads / 32; ++w) mx = max(mx, warp_max[w]);
+    const int E = static_cast<int>(mx >> 7);            // biased exponent of the largest |x|
+    int e = (mx == 0 || E >= 255) ? 0 : E - 142;          // largest |x| * 2^-e in [2^15, 2^16)
+    e = max(-100, min(112, e));
+    const float scale = __int_as_float((127 - e) << 23);  // 2^-e
+    for (int i = threadIdx.x; i < K8; i += kConvThreads) {
+        const uint4 v = src[i];
+        uint4 o;
+        o.x = bf16x2_to_f16x2(v.x, scale);
+        o.y = bf16x2_to_f16x2(v.y, scale);
+        o.z = bf16x2_to_f16x2(v.z, scale);
+        o.w = bf16x2_to_f16x2(v.w, scale);
+        dst[i] = o;
+    }
+    if (threadIdx.x == 0) rowmul[row] = __int_as_float((127 + e) << 23);   // 2^e
 }
 
 // One CTA waits on a barrier that nothing arrives on, with the GEMM's bounded wait: the wait
@@ -541,7 +605,10 @@ lowbit_status launch(const GemmProblem& g, int ksplit_request, cudaStream_t stre
     const CUtensorMapSwizzle wswz = C::kWRowBytes == 16   ? CU_TENSOR_MAP_SWIZZLE_NONE
                                     : C::kWRowBytes == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
                                                           : CU_TENSOR_MAP_SWIZZLE_64B;
-    bool ok = make_map_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.X, K, M, uint64_t(K) * 2, 64, BT,
+    const WorkspaceLayout ws = workspace_layout(g.M, g.K);
+    void* xh = g.workspace;
+    float* rowmul = reinterpret_cast<float*>(static_cast<uint8_t*>(g.workspace) + ws.rowmul_offset);
+    bool ok = make_map_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, xh, K, M, uint64_t(K) * 2, 64, BT,
                           CU_TENSOR_MAP_SWIZZLE_128B);
     ok = ok && make_map_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, g.Wp, uint64_t(K) * BITS / 32, N,
                            uint64_t(K) * BITS / 8, C::kWordsPerRow, kBlockN, wswz);
@@ -563,6 +630,7 @@ lowbit_status launch(const GemmProblem& g, int ksplit_request, cudaStream_t stre
     p.n_tiles = (N + kBlockN - 1) / kBlockN;
     p.num_tiles = p.m_tiles * p.n_tiles;
     p.Y = static_cast<__nv_bfloat16*>(g.Y);
+    p.rowmul = rowmul;
     int ksplit = ksplit_request;
     if (ksplit < 1) ksplit = 1;
     if (ksplit > 8) ksplit = 8;
@@ -571,6 +639,23 @@ lowbit_status launch(const GemmProblem& g, int ksplit_request, cudaStream_t stre
     ksplit = (p.num_kb + kbps - 1) / kbps;     // every rank gets at least one k-block
     p.kb_per_split = ksplit > 1 ? kbps : p.num_kb;
     p.ksplit = ksplit;
+
+    // X -> fp16 copy in the workspace, then the GEMM; both launched as programmatic dependents
+    // of whatever precedes them on the stream.
+    {
+        cudaLaunchConfig_t ccfg = {};
+        cudaLaunchAttribute cattr[1];
+        cattr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        cattr[0].val.programmaticStreamSerializationAllowed = 1;
+        ccfg.gridDim = dim3(M, 1, 1);
+        ccfg.blockDim = dim3(kConvThreads, 1, 1);
+        ccfg.stream = stream;
+        ccfg.attrs = cattr;
+        ccfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&ccfg, convert_x_kernel, static_cast<const uint4*>(g.X), K / 8,
+                               static_cast<uint4*>(xh), rowmul) != cudaSuccess)
+            return LOWBIT_ERR_CUDA;
+    }
 
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attrs[2];

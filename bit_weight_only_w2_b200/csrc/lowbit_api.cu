@@ -58,6 +58,9 @@ lowbit_status validate_gemm(const GemmProblem& g) {
     if (g.N % 8 != 0) return LOWBIT_ERR_UNSUPPORTED;
     if (g.M >= (int64_t(1) << 31) || g.N >= (int64_t(1) << 31) || g.K >= (int64_t(1) << 31))
         return LOWBIT_ERR_UNSUPPORTED;
+    if (!g.workspace || (reinterpret_cast<uintptr_t>(g.workspace) & 255u) != 0 ||
+        g.workspace_bytes < workspace_layout(g.M, g.K).total)
+        return LOWBIT_ERR_WORKSPACE;
     return LOWBIT_OK;
 }
 
@@ -75,6 +78,7 @@ LOWBIT_API const char* lowbit_status_string(lowbit_status s) {
         case LOWBIT_ERR_BAD_CODE: return "LOWBIT_ERR_BAD_CODE";
         case LOWBIT_ERR_TIMEOUT: return "LOWBIT_ERR_TIMEOUT";
         case LOWBIT_ERR_CUDA: return "LOWBIT_ERR_CUDA";
+        case LOWBIT_ERR_WORKSPACE: return "LOWBIT_ERR_WORKSPACE";
     }
     return "LOWBIT_ERR_UNKNOWN";
 }
@@ -111,7 +115,8 @@ LOWBIT_API lowbit_status lowbit_unpack(const uint32_t* packed, int64_t N, int64_
 }
 
 static GemmProblem make_problem(int64_t M, int64_t N, int64_t K, int bits, int group_size, const void* X,
-                                const uint32_t* Wp, const void* scales, const void* zeros, void* Y) {
+                                const uint32_t* Wp, const void* scales, const void* zeros, void* Y,
+                                void* workspace, size_t workspace_bytes) {
     GemmProblem g;
     g.M = M;
     g.N = N;
@@ -123,13 +128,20 @@ static GemmProblem make_problem(int64_t M, int64_t N, int64_t K, int bits, int g
     g.scales = scales;
     g.zeros = zeros;
     g.Y = Y;
+    g.workspace = workspace;
+    g.workspace_bytes = workspace_bytes;
     return g;
+}
+
+LOWBIT_API size_t lowbit_gemm_workspace_size(int64_t M, int64_t K) {
+    if (M < 0 || K < 0) return 0;
+    return workspace_layout(M, K).total;
 }
 
 LOWBIT_API lowbit_status lowbit_gemm(int64_t M, int64_t N, int64_t K, int bits, int group_size, const void* X,
                                      const uint32_t* Wp, const void* scales, const void* zeros, void* Y,
-                                     void* stream) {
-    const GemmProblem g = make_problem(M, N, K, bits, group_size, X, Wp, scales, zeros, Y);
+                                     void* workspace, size_t workspace_bytes, void* stream) {
+    const GemmProblem g = make_problem(M, N, K, bits, group_size, X, Wp, scales, zeros, Y, workspace, workspace_bytes);
     lowbit_status st = validate_gemm(g);
     if (st != LOWBIT_OK || M == 0 || N == 0) return st;
     if ((st = check_device()) != LOWBIT_OK) return st;
@@ -138,8 +150,9 @@ LOWBIT_API lowbit_status lowbit_gemm(int64_t M, int64_t N, int64_t K, int bits, 
 
 LOWBIT_API lowbit_status lowbit_gemm_ex(int64_t M, int64_t N, int64_t K, int bits, int group_size, const void* X,
                                         const uint32_t* Wp, const void* scales, const void* zeros, void* Y,
-                                        int tile_tokens, int ksplit, void* stream) {
-    const GemmProblem g = make_problem(M, N, K, bits, group_size, X, Wp, scales, zeros, Y);
+                                        void* workspace, size_t workspace_bytes, int tile_tokens, int ksplit,
+                                        void* stream) {
+    const GemmProblem g = make_problem(M, N, K, bits, group_size, X, Wp, scales, zeros, Y, workspace, workspace_bytes);
     lowbit_status st = validate_gemm(g);
     if (st != LOWBIT_OK || M == 0 || N == 0) return st;
     if (tile_tokens != 0 && tile_tokens != 16 && tile_tokens != 32 && tile_tokens != 64 && tile_tokens != 128 &&
@@ -150,12 +163,13 @@ LOWBIT_API lowbit_status lowbit_gemm_ex(int64_t M, int64_t N, int64_t K, int bit
     return gemm_launch(g, tile_tokens, ksplit, static_cast<cudaStream_t>(stream));
 }
 
-LOWBIT_API lowbit_status lowbit_gemm_batch(const lowbit_gemm_desc* descs, int count, void* stream) {
+LOWBIT_API lowbit_status lowbit_gemm_batch(const lowbit_gemm_desc* descs, int count, void* workspace,
+                                           size_t workspace_bytes, void* stream) {
     if (count < 0 || (count > 0 && !descs)) return LOWBIT_ERR_INVALID_ARG;
     for (int i = 0; i < count; ++i) {
         const lowbit_gemm_desc& d = descs[i];
-        const lowbit_status st = validate_gemm(
-            make_problem(d.M, d.N, d.K, d.bits, d.group_size, d.X, d.Wp, d.scales, d.zeros, d.Y));
+        const lowbit_status st = validate_gemm(make_problem(d.M, d.N, d.K, d.bits, d.group_size, d.X, d.Wp,
+                                                            d.scales, d.zeros, d.Y, workspace, workspace_bytes));
         if (st != LOWBIT_OK) return st;
     }
     if (count == 0) return LOWBIT_OK;
@@ -164,7 +178,8 @@ LOWBIT_API lowbit_status lowbit_gemm_batch(const lowbit_gemm_desc* descs, int co
     for (int i = 0; i < count; ++i) {
         const lowbit_gemm_desc& d = descs[i];
         if (d.M == 0 || d.N == 0) continue;
-        st = gemm_launch(make_problem(d.M, d.N, d.K, d.bits, d.group_size, d.X, d.Wp, d.scales, d.zeros, d.Y),
+        st = gemm_launch(make_problem(d.M, d.N, d.K, d.bits, d.group_size, d.X, d.Wp, d.scales, d.zeros, d.Y,
+                                      workspace, workspace_bytes),
                          0, 0, static_cast<cudaStream_t>(stream));
         if (st != LOWBIT_OK) return st;
     }

@@ -17,7 +17,20 @@ struct GemmProblem {
     const void* scales;
     const void* zeros;
     void* Y;
+    void* workspace;
+    size_t workspace_bytes;
 };
+
+// Workspace of one GEMM: the fp16 copy of X ([M][K]) then one fp32 factor per row of X.
+struct WorkspaceLayout {
+    size_t rowmul_offset;
+    size_t total;
+};
+inline WorkspaceLayout workspace_layout(int64_t M, int64_t K) {
+    const size_t xh = (static_cast<size_t>(M) * static_cast<size_t>(K) * 2 + 255) / 256 * 256;
+    const size_t rm = (static_cast<size_t>(M) * 4 + 255) / 256 * 256;
+    return WorkspaceLayout{xh, xh + rm};
+}
 
 // Validates one problem against the ABI's preconditions (no launch, no CUDA call).
 lowbit_status validate_gemm(const GemmProblem& g);

@@ -27,10 +27,16 @@
  *   register, so a decoder builds bf16x2 operands with one mask per pair.)
  *
  * Scale / zero layout: fp16, group-major [K/group_size][N]: s(n, k) = scales[(k/g)*N + n].
- * X: bf16 row-major [M][K]. Y: bf16 row-major [M][N]. Accumulation is fp32.
+ * X: bf16 row-major [M][K]. Y: bf16 row-major [M][N].
  *
- * Ownership: the caller owns every buffer (device memory unless stated). The library keeps
- * no allocation; it holds one small status word per device in static device memory.
+ * Arithmetic: X is copied to fp16 in the caller's workspace (exactly: each row is first scaled
+ * by a power of two that keeps it inside fp16's range, and the result is scaled back), weights
+ * are decoded to fp16 (binary / ternary exactly, uint4 with one rounding), products are summed
+ * in fp32 on the tensor cores and Y is rounded to bf16 once.
+ *
+ * Ownership: the caller owns every buffer (device memory unless stated), including the GEMM
+ * workspace (see lowbit_gemm_workspace_size). The library allocates nothing; it holds a few
+ * status words per device in static device memory.
  * Streams are CUDA stream handles (cudaStream_t) passed as void*; NULL = legacy stream.
  * Errors: argument / shape errors return before any launch and change nothing.
  */
@@ -52,7 +58,8 @@ typedef enum lowbit_status {
     LOWBIT_ERR_UNSUPPORTED_DEVICE = 4, /* current device is not sm_100 (B200 class)             */
     LOWBIT_ERR_BAD_CODE = 5,           /* pack: a code outside its format; unpack: field 3       */
     LOWBIT_ERR_TIMEOUT = 6,            /* a bounded wait inside a kernel gave up (device status) */
-    LOWBIT_ERR_CUDA = 7                /* a CUDA runtime / driver call failed                    */
+    LOWBIT_ERR_CUDA = 7,               /* a CUDA runtime / driver call failed                    */
+    LOWBIT_ERR_WORKSPACE = 8           /* workspace NULL, misaligned or smaller than required    */
 } lowbit_status;
 
 /* Human-readable name of a status. Never NULL. */
@@ -78,19 +85,27 @@ lowbit_status lowbit_pack(const int8_t* codes, int64_t N, int64_t K, int bits, u
 lowbit_status lowbit_unpack(const uint32_t* packed, int64_t N, int64_t K, int bits, int8_t* codes,
                             void* stream);
 
-/* Y = X * W^T on `stream` (asynchronous; never synchronises).
- *   X       [M][K]            bf16, device, 16-byte aligned
- *   Wp      [N][K*bits/32]    uint32 packed codes, device, 16-byte aligned
- *   scales  [K/group_size][N] fp16, device, 16-byte aligned
- *   zeros   [K/group_size][N] fp16 for bits == 4, NULL otherwise
- *   Y       [M][N]            bf16, device, 16-byte aligned; must not overlap the inputs
+/* Bytes of device workspace lowbit_gemm needs for an X of [M][K]: the fp16 copy of X
+ * (M*K*2 bytes, rounded up to 256) plus one float per row (rounded up to 256). 0 if M or K < 0. */
+size_t lowbit_gemm_workspace_size(int64_t M, int64_t K);
+
+/* Y = X * W^T on `stream` (asynchronous; never synchronises). Two kernels run in order on the
+ * stream: the X -> fp16 conversion into `workspace`, then the GEMM.
+ *   X          [M][K]            bf16, device, 16-byte aligned
+ *   Wp         [N][K*bits/32]    uint32 packed codes, device, 16-byte aligned
+ *   scales     [K/group_size][N] fp16, device, 16-byte aligned
+ *   zeros      [K/group_size][N] fp16 for bits == 4, NULL otherwise
+ *   Y          [M][N]            bf16, device, 16-byte aligned; must not overlap the inputs
+ *   workspace  device, 256-byte aligned, >= lowbit_gemm_workspace_size(M, K) bytes; owned by
+ *              the caller, overwritten by the call, and must not be used by concurrently
+ *              running work until the call's kernels have finished
  * GPU path preconditions (else LOWBIT_ERR_UNSUPPORTED): group_size 64 or 128,
  * K % group_size == 0, K % 128 == 0 when bits == 1, N % 8 == 0, M, N, K < 2^31.
  * M == 0 or N == 0 is a no-op. Kernel-side bounded waits that give up set the device
  * status word (see lowbit_device_status) instead of trapping. */
 lowbit_status lowbit_gemm(int64_t M, int64_t N, int64_t K, int bits, int group_size, const void* X,
                           const uint32_t* Wp, const void* scales, const void* zeros, void* Y,
-                          void* stream);
+                          void* workspace, size_t workspace_bytes, void* stream);
 
 /* lowbit_gemm with the kernel configuration fixed instead of chosen from the shape, for
  * tuning and tests: `tile_tokens` = tokens per CTA tile (16, 32, 64, 128 or 256; 0 = automatic),
@@ -99,7 +114,8 @@ lowbit_status lowbit_gemm(int64_t M, int64_t N, int64_t K, int bits, int group_s
  * tile_tokens returns LOWBIT_ERR_UNSUPPORTED. */
 lowbit_status lowbit_gemm_ex(int64_t M, int64_t N, int64_t K, int bits, int group_size, const void* X,
                              const uint32_t* Wp, const void* scales, const void* zeros, void* Y,
-                             int tile_tokens, int ksplit, void* stream);
+                             void* workspace, size_t workspace_bytes, int tile_tokens, int ksplit,
+                             void* stream);
 
 /* One linear of a chain, with the meaning and layout of lowbit_gemm's arguments. */
 typedef struct lowbit_gemm_desc {
@@ -113,11 +129,13 @@ typedef struct lowbit_gemm_desc {
 } lowbit_gemm_desc;
 
 /* Run `count` GEMMs (host array of descriptors) in order on `stream`, as if lowbit_gemm were
- * called for each in turn: a descriptor may read an earlier one's Y. All descriptors are
- * validated first; on any invalid one nothing is launched and its error is returned.
- * Consecutive launches overlap their prologues with the previous kernel's tail
+ * called for each in turn with the same workspace: a descriptor may read an earlier one's Y.
+ * The workspace must hold the largest lowbit_gemm_workspace_size(M, K) of the descriptors.
+ * All descriptors are validated first; on any invalid one nothing is launched and its error
+ * is returned. Consecutive launches overlap their prologues with the previous kernel's tail
  * (programmatic dependent launch); results are the same as separate calls. */
-lowbit_status lowbit_gemm_batch(const lowbit_gemm_desc* descs, int count, void* stream);
+lowbit_status lowbit_gemm_batch(const lowbit_gemm_desc* descs, int count, void* workspace,
+                                size_t workspace_bytes, void* stream);
 
 /* Read the current device's sticky status word, written by kernels whose bounded waits gave
  * up (LOWBIT_ERR_TIMEOUT), and clear it when `clear` != 0. Synchronises the device. */

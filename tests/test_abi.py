@@ -30,7 +30,8 @@ def lib():
 def test_header_declares_entry_points():
     names = declared_functions()
     for required in ("lowbit_pack", "lowbit_unpack", "lowbit_gemm", "lowbit_gemm_batch", "lowbit_gemm_ex",
-                     "lowbit_packed_words", "lowbit_device_status", "lowbit_status_string"):
+                     "lowbit_packed_words", "lowbit_device_status", "lowbit_status_string",
+                     "lowbit_gemm_workspace_size"):
         assert required in names
 
 
@@ -49,9 +50,14 @@ def test_host_functions(lib):
     assert lib.lowbit_packed_words(4, 48, 1) == 0      # K not a multiple of 32
     assert lib.lowbit_packed_words(4, 64, 3) == 0      # bits
     assert lib.lowbit_packed_words(-1, 64, 2) == 0
+    assert lib.lowbit_status_string(8) == b"LOWBIT_ERR_WORKSPACE"
+    assert lib.lowbit_gemm_workspace_size(4608, 3072) == 4608 * 3072 * 2 + 4608 * 4
+    assert lib.lowbit_gemm_workspace_size(1, 64) == 256 + 256
+    assert lib.lowbit_gemm_workspace_size(-1, 64) == 0
 
 
-A = 1 << 20  # a fake 16-byte-aligned address: never dereferenced, checks fail first
+A = 1 << 20  # a fake 256-byte-aligned address: never dereferenced, checks fail first
+WS = 1 << 30  # fake workspace size, large enough for every shape below
 
 
 @pytest.mark.parametrize("args,expect", [
@@ -67,19 +73,22 @@ A = 1 << 20  # a fake 16-byte-aligned address: never dereferenced, checks fail f
     (dict(N=100), 3),                       # N % 8
     (dict(bits=1, K=192, group_size=64), 3),  # binary needs K % 128
     (dict(M=-1), 1),
+    (dict(ws=0), 8),                        # no workspace
+    (dict(ws=A + 16), 8),                   # workspace not 256-byte aligned
+    (dict(ws_bytes=16 * 256 * 2), 8),       # too small (row factors missing)
 ])
 def test_gemm_rejects_before_launch(lib, args, expect):
-    a = dict(M=16, N=128, K=256, bits=2, group_size=128, X=A, Wp=A, scales=A, zeros=0, Y=A)
+    a = dict(M=16, N=128, K=256, bits=2, group_size=128, X=A, Wp=A, scales=A, zeros=0, Y=A, ws=A, ws_bytes=WS)
     a.update(args)
     st = lib.lowbit_gemm(a["M"], a["N"], a["K"], a["bits"], a["group_size"], a["X"], a["Wp"], a["scales"],
-                         a["zeros"] or None, a["Y"], None)
+                         a["zeros"] or None, a["Y"], a["ws"] or None, a["ws_bytes"], None)
     assert st == expect, lb.STATUS.get(st)
 
 
 def test_gemm_ex_rejects_bad_tile(lib):
-    st = lib.lowbit_gemm_ex(16, 128, 256, 2, 128, A, A, A, None, A, 48, 0, None)
+    st = lib.lowbit_gemm_ex(16, 128, 256, 2, 128, A, A, A, None, A, A, WS, 48, 0, None)
     assert st == 3
-    st = lib.lowbit_gemm_ex(16, 128, 256, 2, 128, A, A, A, None, A, 16, 9, None)
+    st = lib.lowbit_gemm_ex(16, 128, 256, 2, 128, A, A, A, None, A, A, WS, 16, 9, None)
     assert st == 3
 
 
@@ -87,14 +96,15 @@ def test_batch_validates_all_first(lib):
     good = lb.GemmDesc(16, 128, 256, 2, 128, A, A, A, None, A)
     bad = lb.GemmDesc(16, 128, 256, 3, 128, A, A, A, None, A)
     arr = (lb.GemmDesc * 2)(good, bad)
-    assert lib.lowbit_gemm_batch(arr, 2, None) == 1
-    assert lib.lowbit_gemm_batch(None, -1, None) == 1
-    assert lib.lowbit_gemm_batch(None, 0, None) == 0
+    assert lib.lowbit_gemm_batch(arr, 2, A, WS, None) == 1
+    assert lib.lowbit_gemm_batch(arr, 1, A, 1024, None) == 8      # workspace too small for the first
+    assert lib.lowbit_gemm_batch(None, -1, A, WS, None) == 1
+    assert lib.lowbit_gemm_batch(None, 0, None, 0, None) == 0
 
 
 def test_empty_problems_are_noops(lib):
-    assert lib.lowbit_gemm(0, 128, 256, 2, 128, A, A, A, None, A, None) == 0
-    assert lib.lowbit_gemm(16, 0, 256, 2, 128, A, A, A, None, A, None) == 0
+    assert lib.lowbit_gemm(0, 128, 256, 2, 128, A, A, A, None, A, None, 0, None) == 0
+    assert lib.lowbit_gemm(16, 0, 256, 2, 128, A, A, A, None, A, None, 0, None) == 0
     assert lib.lowbit_pack(None, 0, 64, 2, None, None) == 0
 
 

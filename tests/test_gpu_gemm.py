@@ -213,3 +213,26 @@ def test_bounded_wait_timeout_is_reported():
     assert lb.device_status(clear=True) == 6
     assert lb.device_status() == 0
     run_and_compare(spec_for(2, 128, 64, 256, 128, seed=1))
+
+
+def test_extreme_row_magnitudes():
+    """Rows far outside fp16's range (huge, tiny, zero, near the bf16 maximum) still match the
+    oracle row by row: X is converted with a per-row power-of-two factor."""
+    spec = spec_for(2, 128, 64, 512, 256, seed=31)
+    prob = synth.make_problem(spec)
+    x = _pins.x_as_f64(prob.x_bf16)
+    x[0] *= 2.0 ** 20
+    x[1] *= 2.0 ** -30
+    x[2] = 0.0
+    x[3] *= 2.0 ** -120
+    x[4, 7] = 3.0e38
+    x[5] *= 2.0 ** 60
+    prob.x_bf16 = _pins.bf16_bits_from_f32(x.astype(np.float32))
+    ref = oracle.gemm(prob.x_bf16, _gpu.oracle_packed(prob), prob.scales, None, spec.N, 2, 128)
+    xd, packed, s, z = _gpu.dev_problem(prob)
+    y = _gpu.y_to_f64(lb.gemm(xd, packed, s, z, 2, 128))
+    assert np.all(y[2] == 0.0)
+    for m in range(spec.M):
+        if m == 2:
+            continue
+        _gpu.check_close(y[m], ref[m], what=f"row {m}")
