@@ -133,4 +133,6 @@ WORKLOADS = {
     ],
     # one denoise step's 80 ternary linears at a 1024x1024 image
     "klein_step_chain_1024sq_ternary_g128": chain_linears(),
+    # its largest linear on its own: a single-stream block's fused QKV + MLP-in (profiling case)
+    "klein_single_qkv_mlp_in_1024sq_ternary_g128": [chain_linears()[40]],
 }

@@ -224,8 +224,8 @@ def test_extreme_row_magnitudes():
     x[0] *= 2.0 ** 20
     x[1] *= 2.0 ** -30
     x[2] = 0.0
-    x[3] *= 2.0 ** -120
-    x[4, 7] = 3.0e38
+    x[3] *= 2.0 ** -100
+    x[4, 7] = 1.5 * 2.0 ** 127          # near the bf16 maximum
     x[5] *= 2.0 ** 60
     prob.x_bf16 = _pins.bf16_bits_from_f32(x.astype(np.float32))
     ref = oracle.gemm(prob.x_bf16, _gpu.oracle_packed(prob), prob.scales, None, spec.N, 2, 128)
