@@ -141,6 +141,31 @@ lowbit_status lowbit_gemm_batch(const lowbit_gemm_desc* descs, int count, void* 
  * up (LOWBIT_ERR_TIMEOUT), and clear it when `clear` != 0. Synchronises the device. */
 lowbit_status lowbit_device_status(int clear);
 
+/* Size of the static device scratch used by lowbit_gemm_noalloc: 32 MiB. */
+#define LOWBIT_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+
+/* lowbit_gemm for callers that cannot allocate device memory where they run a linear -- for
+ * example a plug-in inside a host engine that owns all device memory and forbids allocations
+ * after start-up, or a latency-critical loop in which cudaMalloc's device synchronisation is not
+ * acceptable. It takes the same arguments as lowbit_gemm minus the workspace: its scratch (the
+ * fp16 copy of X and the row factors) lives in a fixed array of static device memory of
+ * LOWBIT_NOALLOC_SCRATCH_BYTES, which a device holds from the first use of this entry point
+ * on it (or from library load, if CUDA modules are loaded eagerly) until the process exits.
+ *  - Problems with lowbit_gemm_workspace_size(M, K) > LOWBIT_NOALLOC_SCRATCH_BYTES (for
+ *    example M * K > about 16.7 million at small M) are rejected with LOWBIT_ERR_WORKSPACE
+ *    before any launch; other argument errors are those of lowbit_gemm.
+ *  - The first call on a device looks up the array's device address (cudaGetSymbolAddress)
+ *    with that device current; make that first call before any stream capture.
+ *  - Nothing in the scratch has to start at zero: each call overwrites the part it reads.
+ *  - All calls on a device share the one array, so calls whose kernels overlap on the GPU
+ *    (different streams or host threads without ordering) race; order them on one stream, or
+ *    use lowbit_gemm with separate workspaces.
+ *  - Allocates nothing: no cudaMalloc / cudaFree and no allocating library routine.
+ * The pages have no counterpart to this entry point; it is a deployment variant of lowbit_gemm. */
+lowbit_status lowbit_gemm_noalloc(int64_t M, int64_t N, int64_t K, int bits, int group_size, const void* X,
+                                  const uint32_t* Wp, const void* scales, const void* zeros, void* Y,
+                                  void* stream);
+
 /* Diagnostic for the kernels' failure detection: launches one CTA that waits on a
  * shared-memory barrier nothing ever completes, using the same bounded wait as the GEMM kernel
  * but giving up after `limit_cycles` SM clocks (> 0). The wait then records LOWBIT_ERR_TIMEOUT in
