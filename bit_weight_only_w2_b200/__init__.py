@@ -66,7 +66,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.lowbit_gemm_workspace_size.restype = sz
     lib.lowbit_gemm.argtypes = [i64, i64, i64, i32, i32, p, p, p, p, p, p, sz, p]
     lib.lowbit_gemm.restype = i32
-    lib.lowbit_gemm_ex.argtypes = [i64, i64, i64, i32, i32, p, p, p, p, p, p, sz, i32, i32, p]
+    lib.lowbit_gemm_ex.argtypes = [i64, i64, i64, i32, i32, p, p, p, p, p, p, sz, i32, i32, i32, p]
     lib.lowbit_gemm_ex.restype = i32
     lib.lowbit_gemm_batch.argtypes = [ctypes.POINTER(GemmDesc), i32, p, sz, p]
     lib.lowbit_gemm_batch.restype = i32
@@ -146,7 +146,7 @@ def workspace(device: torch.device, nbytes: int) -> torch.Tensor:
 
 def gemm(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, zeros: Optional[torch.Tensor],
          bits: int, group_size: int, out: Optional[torch.Tensor] = None, tile_tokens: int = 0,
-         ksplit: int = 0, ws: Optional[torch.Tensor] = None) -> torch.Tensor:
+         ksplit: int = 0, ws: Optional[torch.Tensor] = None, tile_rows: int = 0) -> torch.Tensor:
     """Y[M][N] = X[M][K] * W^T with W decoded from `packed`, `scales` (and `zeros`)."""
     _need(x, torch.bfloat16, "x")
     _need(packed, torch.int32, "packed")
@@ -164,9 +164,9 @@ def gemm(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, zeros: Opt
         need = workspace_size(M, K)
         if ws is None:
             ws = workspace(x.device, need)
-        if tile_tokens or ksplit:
+        if tile_tokens or ksplit or tile_rows:
             st = lib.lowbit_gemm_ex(M, N, K, bits, group_size, _ptr(x), _ptr(packed), _ptr(scales), _ptr(zeros),
-                                    _ptr(out), _ptr(ws), ws.numel(), tile_tokens, ksplit, _stream(x))
+                                    _ptr(out), _ptr(ws), ws.numel(), tile_tokens, tile_rows, ksplit, _stream(x))
         else:
             st = lib.lowbit_gemm(M, N, K, bits, group_size, _ptr(x), _ptr(packed), _ptr(scales), _ptr(zeros),
                                  _ptr(out), _ptr(ws), ws.numel(), _stream(x))

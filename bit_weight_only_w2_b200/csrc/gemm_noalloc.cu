@@ -70,5 +70,5 @@ LOWBIT_API lowbit_status lowbit_gemm_noalloc(int64_t M, int64_t N, int64_t K, in
     if (st != LOWBIT_OK || M == 0 || N == 0) return st;
     if ((st = check_device()) != LOWBIT_OK) return st;
     if ((st = scratch_address(&g.workspace)) != LOWBIT_OK) return st;
-    return gemm_launch(g, 0, 0, static_cast<cudaStream_t>(stream));
+    return gemm_launch(g, 0, 0, 0, static_cast<cudaStream_t>(stream));
 }

@@ -17,10 +17,11 @@
 // break a 1e-2 tolerance in the tails.
 //
 // Kernel design ("swap AB", weights as the MMA's A operand):
-//   * One CTA tile = 128 weight rows (MMA M) x BT tokens (MMA N), K in stages of 128.
+//   * One CTA tile = up to 128 weight rows (MMA M) x BT tokens (MMA N), K in stages of 128.
 //   * Warp 0 (one lane) is the TMA producer: per stage it loads two 64-wide, 128B-swizzled
-//     boxes of the fp16 copy of X (the MMA's B operand, K-major), the packed code box of the 128 rows and their
-//     group scales (and zeros) into a shared-memory ring.
+//     boxes of the fp16 copy of X (the MMA's B operand, K-major), the packed code box of the
+//     tile's rows and their group scales (and zeros) into a shared-memory ring. The first
+//     stages' weight boxes are requested before waiting for the X conversion to finish.
 //   * The dequant warps each own 32 weight rows (one per lane, matching the tensor-memory lane
 //     quarter the warp may access): they read the row's packed words from shared memory,
 //     decode codes x scale to fp16 pairs with a few integer / fp16x2 instructions per pair,
@@ -28,12 +29,14 @@
 //     never touch shared memory, which leaves its bandwidth to TMA and the MMA's B reads.
 //   * Warp 1 (one lane) issues tcgen05.mma (kind::f16, A from tensor memory, B from shared
 //     memory, fp32 accumulators in tensor memory) and frees ring slots with tcgen05.commit.
-//   * Four epilogue warps read the accumulators with tcgen05.ld, apply the row's power-of-two
-//     scale, round to bf16 and store Y.
-//     With two accumulator buffers the epilogue of one tile overlaps the next tile's MMAs.
-//   * Without split-K the grid is persistent (tiles strided over the CTAs). With split-K
-//     (small M, few tiles) the K range is divided over the CTAs of a thread-block cluster and
-//     the fp32 partial tiles are summed in a fixed order through distributed shared memory.
+//   * Epilogue warps (8 for 128/256-token tiles) read the accumulators with tcgen05.ld, apply
+//     the row's power-of-two factor, round to bf16 into registers and hand the accumulator
+//     back before storing, so a tile's stores overlap the next tile's MMAs even with a single
+//     accumulator buffer; neighbouring lanes swap halves so each store writes two outputs.
+//   * Grids: persistent over 128-row tiles when there are many; for small M either "flat"
+//     tiles of ceil(N / #SMs) rows with the whole K per CTA, or K split over the CTAs of a
+//     thread-block cluster whose fp32 partial tiles are summed in rank order through
+//     distributed shared memory.
 //   * Every mbarrier wait is bounded (see sm100_ptx.cuh): a wait that gives up records
 //     LOWBIT_ERR_TIMEOUT in the device status word and the CTA drains and exits.
 #include <cuda.h>
@@ -52,10 +55,9 @@ namespace lowbit {
 
 __device__ unsigned g_device_status = 0;
 
-constexpr int kBlockN = 128;        // weight rows per tile (MMA M)
+constexpr int kBlockN = 128;        // weight rows per tile at most (MMA M)
 constexpr int kBlockK = 128;        // K per pipeline stage
-constexpr int kNumCtrlWarps = 4;    // warp 0: TMA, warp 1: MMA + TMEM owner, warps 2-3 idle
-constexpr int kNumEpiWarps = 4;
+constexpr int kNumCtrlWarps = 2;    // warp 0: TMA producer, warp 1: MMA issuer + TMEM owner
 constexpr int kSmemLimit = 232448;  // 227 KB opt-in dynamic shared memory per block
 
 template <int BITS, int GS, int BT>
@@ -64,10 +66,16 @@ struct Cfg {
     static_assert(GS == 64 || GS == 128, "group size");
     static_assert(BT % 16 == 0 && BT >= 16 && BT <= 256, "MMA N");
     static constexpr int kCtasPerSm = (BT <= 64) ? 2 : 1;
+    // Epilogue: warps e and e+4 cover the same 32 weight rows (TMEM lane quarter = warp % 4),
+    // each half of the tile's token columns when there are 8.
+    static constexpr int kNumEpiWarps = (BT >= 128) ? 8 : 4;
+    static constexpr int kEpiParts = kNumEpiWarps / 4;
+    static constexpr int kEpiCols = BT / kEpiParts;                 // accumulator columns per thread
     static constexpr int kNumDqWarps = (BITS == 4) ? 8 : 4;
-    static constexpr int kParts = kNumDqWarps / 4;                 // dequant warps per row quarter
-    static constexpr int kThreads = 32 * (kNumCtrlWarps + kNumEpiWarps + kNumDqWarps);
+    static constexpr int kParts = kNumDqWarps / 4;                  // dequant warps per row quarter
+    static constexpr int kFirstEpiWarp = kNumCtrlWarps;
     static constexpr int kFirstDqWarp = kNumCtrlWarps + kNumEpiWarps;
+    static constexpr int kThreads = 32 * (kNumCtrlWarps + kNumEpiWarps + kNumDqWarps);
     static constexpr int kNumAcc = (BT == 64 || BT == 256) ? 1 : 2;   // fit the tensor-memory budget
     static constexpr int kAccCols = kNumAcc * BT;
     static constexpr int kACol0 = (kAccCols + 31) / 32 * 32;
@@ -90,7 +98,7 @@ struct Cfg {
     static constexpr int kSOff = kWOff + kWBytes;
     static constexpr int kZOff = kSOff + kSBytes;
     static constexpr int kStageBytes = (kZOff + kZBytes + 1023) / 1024 * 1024;
-    static constexpr int kTxBytes = kXBytes + kWBytes + kSBytes + kZBytes;
+    static constexpr int kTxFixed = kXBytes + kSBytes + kZBytes;   // plus rows * kWRowBytes
     static constexpr int kBarBytes = 1024;
     static constexpr int kBudget = kSmemLimit / kCtasPerSm - 1024 /*align*/ - kBarBytes - 2048 /*reserve*/;
     static constexpr int kStagesFit = kBudget / kStageBytes;
@@ -103,8 +111,9 @@ struct Cfg {
     static constexpr int kSmemFloor = (kCtasPerSm == 2) ? 80 * 1024 : 150 * 1024;
     static constexpr int kSmemBytes = kSmemNeeded > kSmemFloor ? kSmemNeeded : kSmemFloor;
     static_assert(kSmemBytes <= kSmemLimit, "shared memory");
-    // split-K partial tile (fp32 [BT][128]) reuses the stage ring
+    // split-K partial tile (fp32 [128][BT], rows of 16-byte chunks XOR-swizzled) reuses the ring
     static_assert(BT * kBlockN * 4 <= kStages * kStageBytes, "split-K partial buffer");
+    static constexpr int kPartSwizzle = (BT / 4 >= 8) ? 7 : (BT / 4 - 1);
     static constexpr uint32_t kIdesc = idesc_f16_f32(kBlockN, BT);
 };
 
@@ -112,8 +121,10 @@ struct KernelParams {
     int M, N, K;
     int num_kb;          // k-blocks of 128
     int kb_per_split;    // k-blocks per cluster rank (split-K), else num_kb
+    int rows;            // weight rows per tile: 128, or fewer (multiple of 8) for small M
     int m_tiles, n_tiles, num_tiles;
-    int ksplit;          // cluster size along z (1 = persistent, no split)
+    int ksplit;          // cluster size along z (1 = no split)
+    uint32_t tx_bytes;   // bytes delivered into one pipeline stage
     __nv_bfloat16* Y;
     const float* rowmul; // per-row power-of-two factor written by the X conversion pass
 };
@@ -208,7 +219,7 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT>::kThreads, Cfg<BITS, GS, BT>
         }
         for (int i = 0; i < NACC; ++i) {
             mbar_init(&accfull[i], 1);
-            mbar_init(&accempty[i], kNumEpiWarps);
+            mbar_init(&accempty[i], C::kNumEpiWarps);
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -229,40 +240,69 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT>::kThreads, Cfg<BITS, GS, BT>
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
 
-    // Wait for the previous kernel in the stream (programmatic dependent launch), then let
-    // the next one start its prologue as soon as SMs free up.
-    grid_dependency_wait();
+    // Programmatic dependent launch: the next kernel in the stream may start its prologue now.
+    // Threads that touch global memory wait for the previous kernel (the X conversion) first.
     grid_launch_dependents();
 
     const bool split = p.ksplit > 1;
     const int kb_begin = split ? static_cast<int>(blockIdx.z) * p.kb_per_split : 0;
     const int kb_end = split ? min(p.num_kb, kb_begin + p.kb_per_split) : p.num_kb;
+    const int nkb = kb_end - kb_begin;
     const int tile_step = split ? p.num_tiles : static_cast<int>(gridDim.x);
+    const int my_tiles =
+        static_cast<int>(blockIdx.x) < p.num_tiles ? (p.num_tiles - 1 - static_cast<int>(blockIdx.x)) / tile_step + 1 : 0;
     unsigned* status = &g_device_status;
 
     if (warp == 0) {
         // ---------------------------------------------------------------- TMA producer
         if (lane == 0) {
-            uint32_t it = 0;
+            const uint32_t total = static_cast<uint32_t>(my_tiles * nkb);
+            auto coords = [&](uint32_t it, int& m0, int& n0, int& kb) {
+                const int tile = static_cast<int>(blockIdx.x) + static_cast<int>(it / nkb) * tile_step;
+                kb = kb_begin + static_cast<int>(it % nkb);
+                m0 = (tile / p.n_tiles) * BT;
+                n0 = (tile % p.n_tiles) * p.rows;
+            };
+            auto load_weights = [&](uint32_t it) {
+                int m0, n0, kb;
+                coords(it, m0, n0, kb);
+                const uint32_t s = it % S;
+                uint8_t* st = smem + s * C::kStageBytes;
+                mbar_arrive_expect_tx(&full[s], p.tx_bytes);
+                tma_load_2d(&map_w, &full[s], st + C::kWOff, kb * C::kWordsPerRow, n0);
+                tma_load_2d(&map_s, &full[s], st + C::kSOff, n0, kb * C::kGroupsPerStage);
+                if (BITS == 4) tma_load_2d(&map_z, &full[s], st + C::kZOff, n0, kb * C::kGroupsPerStage);
+            };
+            auto load_x = [&](uint32_t it) {
+                int m0, n0, kb;
+                coords(it, m0, n0, kb);
+                const uint32_t s = it % S;
+                uint8_t* st = smem + s * C::kStageBytes;
+                tma_load_2d(&map_x, &full[s], st + C::kXOff, kb * kBlockK, m0);
+                tma_load_2d(&map_x, &full[s], st + C::kXOff + C::kXHalfBytes, kb * kBlockK + 64, m0);
+            };
+            // The packed weights and scales are not written by the kernel just before this one
+            // (the X conversion, which itself starts only once everything earlier in the stream
+            // has completed), so the first stages' weight boxes are requested before waiting for
+            // it; their X boxes follow as soon as the conversion is done.
+            const uint32_t pre = total < static_cast<uint32_t>(S) ? total : static_cast<uint32_t>(S);
+            for (uint32_t it = 0; it < pre; ++it) load_weights(it);
+            grid_dependency_wait();
+            for (uint32_t it = 0; it < pre; ++it) load_x(it);
+            uint32_t it = pre;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += tile_step) {
-                const int m0 = (tile / p.n_tiles) * BT;
-                const int n0 = (tile % p.n_tiles) * kBlockN;
-                for (int kb = kb_begin; kb < kb_end; ++kb, ++it) {
-                    const uint32_t s = it % S, ph = (it / S) & 1u;
-                    if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, status)) { ok = false; break; }
-                    uint8_t* st = smem + s * C::kStageBytes;
-                    mbar_arrive_expect_tx(&full[s], C::kTxBytes);
-                    tma_load_2d(&map_x, &full[s], st + C::kXOff, kb * kBlockK, m0);
-                    tma_load_2d(&map_x, &full[s], st + C::kXOff + C::kXHalfBytes, kb * kBlockK + 64, m0);
-                    tma_load_2d(&map_w, &full[s], st + C::kWOff, kb * C::kWordsPerRow, n0);
-                    tma_load_2d(&map_s, &full[s], st + C::kSOff, n0, kb * C::kGroupsPerStage);
-                    if (BITS == 4) tma_load_2d(&map_z, &full[s], st + C::kZOff, n0, kb * C::kGroupsPerStage);
+            for (; it < total; ++it) {
+                const uint32_t s = it % S, ph = (it / S) & 1u;
+                if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, status)) {
+                    ok = false;
+                    break;
                 }
+                load_weights(it);
+                load_x(it);
             }
             if (!ok) {
                 // Drain: wait (bounded) for the copies still in flight before the CTA exits.
-                for (uint32_t j = (it > (uint32_t)S ? it - S : 0u); j < it; ++j) {
+                for (uint32_t j = (it > static_cast<uint32_t>(S) ? it - S : 0u); j < it; ++j) {
                     const long long t0 = clock64();
                     while (!mbar_try_wait(&full[j % S], (j / S) & 1u) && clock64() - t0 < kWaitLimitCycles) {
                     }
@@ -275,9 +315,12 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT>::kThreads, Cfg<BITS, GS, BT>
             uint32_t it = 0, ait = 0, tcount = 0;
             bool ok = true;
             bool issued = false;
-            for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += tile_step, ++tcount) {
+            for (int t = 0; t < my_tiles && ok; ++t, ++tcount) {
                 const uint32_t b = tcount % NACC, acc_ph = (tcount / NACC) & 1u;
-                if (!mbar_wait(&accempty[b], acc_ph ^ 1u, abort_flag, status)) { ok = false; break; }
+                if (!mbar_wait(&accempty[b], acc_ph ^ 1u, abort_flag, status)) {
+                    ok = false;
+                    break;
+                }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + b * BT;
                 for (int kb = kb_begin; kb < kb_end; ++kb, ++it, ++ait) {
@@ -315,55 +358,57 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT>::kThreads, Cfg<BITS, GS, BT>
         const int quarter = warp & 3;
         const int part = dq >> 2;                    // which K part of the stage this warp decodes
         const int row = quarter * 32 + lane;         // weight row within the tile = TMEM lane
+        const bool row_ok = row < p.rows;
         const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
         constexpr int kHalvesPerPart = 2 / C::kParts;   // 64-wide K halves decoded by this warp
         uint32_t it = 0, ait = 0;
         bool ok = true;
-        for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += tile_step) {
+        for (int t = 0; t < my_tiles && ok; ++t) {
             for (int kb = kb_begin; kb < kb_end; ++kb, ++it, ++ait) {
                 const uint32_t s = it % S, ph = (it / S) & 1u;
                 const uint32_t a = ait % NA, aph = (ait / NA) & 1u;
                 if (!__all_sync(0xffffffffu, mbar_wait(&full[s], ph, abort_flag, status))) { ok = false; break; }
                 const uint8_t* st = smem + s * C::kStageBytes;
-                // --- read this row's packed words and scales from shared memory
+                // --- this row's packed words and scales (rows past the tile decode to zero)
                 uint32_t words[kHalvesPerPart][C::kWordsPerRow / 2];
+                uint32_t s2[kHalvesPerPart], c2[kHalvesPerPart];
                 const uint8_t* wrow = st + C::kWOff + row * C::kWRowBytes;
 #pragma unroll
                 for (int hh = 0; hh < kHalvesPerPart; ++hh) {
                     const int h = part * kHalvesPerPart + hh;
-                    if (BITS == 1) {
-                        const uint2 v = *reinterpret_cast<const uint2*>(wrow + h * 8);
-                        words[hh][0] = v.x;
-                        words[hh][1] = v.y;
-                    } else if (BITS == 2) {
-                        const int chunk = h ^ ((row >> 2) & 1);           // 32-byte swizzle
-                        const uint4 v = *reinterpret_cast<const uint4*>(wrow + chunk * 16);
-                        words[hh][0] = v.x; words[hh][1] = v.y; words[hh][2] = v.z; words[hh][3] = v.w;
-                    } else {
-#pragma unroll
-                        for (int q = 0; q < 2; ++q) {
-                            const int chunk = (2 * h + q) ^ ((row >> 1) & 3);  // 64-byte swizzle
-                            const uint4 v = *reinterpret_cast<const uint4*>(wrow + chunk * 16);
-                            words[hh][4 * q + 0] = v.x; words[hh][4 * q + 1] = v.y;
-                            words[hh][4 * q + 2] = v.z; words[hh][4 * q + 3] = v.w;
-                        }
-                    }
-                }
-                uint32_t s2[kHalvesPerPart], c2[kHalvesPerPart];
-#pragma unroll
-                for (int hh = 0; hh < kHalvesPerPart; ++hh) {
-                    const int h = part * kHalvesPerPart + hh;
                     const int gi = (GS == 64) ? h : 0;
-                    const uint16_t* srow = reinterpret_cast<const uint16_t*>(st + C::kSOff) + gi * kBlockN;
-                    const uint32_t sb = srow[row];
-                    s2[hh] = sb | (sb << 16);
-                    if (BITS == 4) {
-                        const __half* zrow = reinterpret_cast<const __half*>(st + C::kZOff) + gi * kBlockN;
-                        const float cz = -__half2float(zrow[row]) * __half2float(__ushort_as_half(static_cast<unsigned short>(sb)));
-                        const uint32_t cb = __half_as_ushort(__float2half_rn(cz));
-                        c2[hh] = cb | (cb << 16);
-                    } else {
-                        c2[hh] = 0;
+#pragma unroll
+                    for (int w = 0; w < C::kWordsPerRow / 2; ++w) words[hh][w] = 0;
+                    s2[hh] = 0;
+                    c2[hh] = 0;
+                    if (row_ok) {
+                        if (BITS == 1) {
+                            const uint2 v = *reinterpret_cast<const uint2*>(wrow + h * 8);
+                            words[hh][0] = v.x;
+                            words[hh][1] = v.y;
+                        } else if (BITS == 2) {
+                            const int chunk = h ^ ((row >> 2) & 1);           // 32-byte swizzle
+                            const uint4 v = *reinterpret_cast<const uint4*>(wrow + chunk * 16);
+                            words[hh][0] = v.x; words[hh][1] = v.y; words[hh][2] = v.z; words[hh][3] = v.w;
+                        } else {
+#pragma unroll
+                            for (int q = 0; q < 2; ++q) {
+                                const int chunk = (2 * h + q) ^ ((row >> 1) & 3);  // 64-byte swizzle
+                                const uint4 v = *reinterpret_cast<const uint4*>(wrow + chunk * 16);
+                                words[hh][4 * q + 0] = v.x; words[hh][4 * q + 1] = v.y;
+                                words[hh][4 * q + 2] = v.z; words[hh][4 * q + 3] = v.w;
+                            }
+                        }
+                        const uint16_t* srow = reinterpret_cast<const uint16_t*>(st + C::kSOff) + gi * kBlockN;
+                        const uint32_t sb = srow[row];
+                        s2[hh] = sb | (sb << 16);
+                        if (BITS == 4) {
+                            const __half* zrow = reinterpret_cast<const __half*>(st + C::kZOff) + gi * kBlockN;
+                            const float cz = -__half2float(zrow[row]) *
+                                             __half2float(__ushort_as_half(static_cast<unsigned short>(sb)));
+                            const uint32_t cb = __half_as_ushort(__float2half_rn(cz));
+                            c2[hh] = cb | (cb << 16);
+                        }
                     }
                 }
                 __syncwarp();
@@ -395,70 +440,133 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT>::kThreads, Cfg<BITS, GS, BT>
                 if (lane == 0) mbar_arrive(&afull[a]);
             }
         }
-    } else if (warp >= kNumCtrlWarps && warp < kNumCtrlWarps + kNumEpiWarps) {
+    } else {
         // ---------------------------------------------------------------- epilogue warps
+        const int e = warp - C::kFirstEpiWarp;
         const int quarter = warp & 3;
+        const int epart = e >> 2;                    // which slice of the token columns
+        const int col0 = epart * C::kEpiCols;
         const int row = quarter * 32 + lane;
+        const bool row_ok = row < p.rows;
         const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
+        grid_dependency_wait();                      // before the first global access
+        constexpr int kChunk = (C::kEpiCols >= 32) ? 32 : 16;
         uint32_t tcount = 0;
-        for (int tile = blockIdx.x; tile < p.num_tiles; tile += tile_step, ++tcount) {
+        for (int t = 0; t < my_tiles; ++t, ++tcount) {
+            const int tile = static_cast<int>(blockIdx.x) + t * tile_step;
             const uint32_t b = tcount % NACC, acc_ph = (tcount / NACC) & 1u;
             if (!__all_sync(0xffffffffu, mbar_wait(&accfull[b], acc_ph, abort_flag, status))) break;
             tc_fence_after();
-            const int m0 = (tile / p.n_tiles) * BT;
-            const int n = (tile % p.n_tiles) * kBlockN + row;
-            constexpr int kChunk = (BT >= 32) ? 32 : 16;
-#pragma unroll 1
-            for (int c0 = 0; c0 < BT; c0 += kChunk) {
-                uint32_t v[32];
-                if (kChunk == 32) {
-                    tmem_ld32(lane_base + b * BT + c0, v);
-                } else {
-                    tmem_ld16(lane_base + b * BT + c0, *reinterpret_cast<uint32_t(*)[16]>(v));
-                }
-                tmem_wait_ld();
-                if (!split) {
-                    // lane j holds the power-of-two factor of token m0 + c0 + j
-                    const int mj = m0 + c0 + lane;
-                    const float mul_j = (lane < kChunk && mj < p.M) ? p.rowmul[mj] : 1.0f;
+            const int m0 = (tile / p.n_tiles) * BT + col0;   // first token of this thread's columns
+            const int n = (tile % p.n_tiles) * p.rows + row;
+            if (!split) {
+                // Read the whole slice into registers (scaled, rounded to bf16), hand the
+                // accumulator back to the MMA issuer, then store: the stores of this tile
+                // overlap the next tile's MMAs.
+                uint32_t packed[C::kEpiCols / 2];
 #pragma unroll
-                    for (int j = 0; j < kChunk; ++j) {
-                        const int m = m0 + c0 + j;
-                        const float mul = __shfl_sync(0xffffffffu, mul_j, j);
-                        if (n < p.N && m < p.M)
-                            p.Y[static_cast<size_t>(m) * p.N + n] = __float2bfloat16_rn(__uint_as_float(v[j]) * mul);
+                for (int c0 = 0; c0 < C::kEpiCols; c0 += kChunk) {
+                    uint32_t v[32];
+                    if (kChunk == 32) {
+                        tmem_ld32(lane_base + b * BT + col0 + c0, v);
+                    } else {
+                        tmem_ld16(lane_base + b * BT + col0 + c0, *reinterpret_cast<uint32_t(*)[16]>(v));
                     }
-                } else {
-                    float* part = reinterpret_cast<float*>(smem);
+                    const int mj = m0 + c0 + lane;           // lane j fetches token m0 + c0 + j's factor
+                    const float mul_j = (lane < kChunk && mj < p.M) ? p.rowmul[mj] : 1.0f;
+                    tmem_wait_ld();
 #pragma unroll
-                    for (int j = 0; j < kChunk; ++j) part[(c0 + j) * kBlockN + row] = __uint_as_float(v[j]);
+                    for (int j = 0; j < kChunk; j += 2) {
+                        const float f0 = __uint_as_float(v[j]) * __shfl_sync(0xffffffffu, mul_j, j);
+                        const float f1 = __uint_as_float(v[j + 1]) * __shfl_sync(0xffffffffu, mul_j, j + 1);
+                        const __nv_bfloat162 h2 = __floats2bfloat162_rn(f0, f1);   // (token j, token j+1)
+                        packed[(c0 + j) / 2] = *reinterpret_cast<const uint32_t*>(&h2);
+                    }
                 }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&accempty[b]);
+                // Lanes 2i and 2i+1 hold rows n and n+1: one shuffle turns each lane's
+                // (token m, token m+1) pair into a 4-byte (row n, row n+1) store at one token.
+                const bool even = (lane & 1) == 0;
+                const int n_pair = even ? n : n - 1;
+                const bool pair_ok = row_ok && (n_pair + 1 < p.N + 1) && n_pair < p.N;
+#pragma unroll
+                for (int j = 0; j < C::kEpiCols; j += 2) {
+                    const uint32_t mine = packed[j / 2];
+                    const uint32_t other = __shfl_xor_sync(0xffffffffu, mine, 1);
+                    const uint32_t outw = even ? __byte_perm(mine, other, 0x5410) : __byte_perm(other, mine, 0x7632);
+                    const int m = m0 + j + (even ? 0 : 1);
+                    if (pair_ok && m < p.M)
+                        *reinterpret_cast<uint32_t*>(p.Y + static_cast<size_t>(m) * p.N + n_pair) = outw;
+                }
+            } else {
+                // split-K: this CTA's fp32 partial goes to shared memory, rows of 16-byte chunks
+                // XOR-swizzled by row so that both the writes and the cluster reads are conflict-free
+                float* part = reinterpret_cast<float*>(smem);
+#pragma unroll
+                for (int c0 = 0; c0 < C::kEpiCols; c0 += kChunk) {
+                    uint32_t v[32];
+                    if (kChunk == 32) {
+                        tmem_ld32(lane_base + b * BT + col0 + c0, v);
+                    } else {
+                        tmem_ld16(lane_base + b * BT + col0 + c0, *reinterpret_cast<uint32_t(*)[16]>(v));
+                    }
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < kChunk; j += 4) {
+                        const int c4 = (col0 + c0 + j) >> 2;
+                        const int pc = c4 ^ (row & C::kPartSwizzle);
+                        *reinterpret_cast<float4*>(part + row * BT + pc * 4) =
+                            make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]), __uint_as_float(v[j + 2]),
+                                        __uint_as_float(v[j + 3]));
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&accempty[b]);
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&accempty[b]);
         }
     }
 
     __syncwarp();
     if (split) {
-        // Sum the K-slices of the cluster in rank order; rank r reduces columns c = r mod ksplit.
+        // Sum the K-slices of the cluster in rank order. Rank r reduces a contiguous range of the
+        // tile's token columns (multiples of 4), read as 16-byte chunks from every rank.
         cluster_sync_all();
-        if (warp >= kNumCtrlWarps && warp < kNumCtrlWarps + kNumEpiWarps && !*abort_flag) {
-            const int row = (warp & 3) * 32 + lane;
+        if (warp >= C::kFirstEpiWarp && warp < C::kFirstDqWarp && !*abort_flag) {
+            const int e = warp - C::kFirstEpiWarp;
+            const int quarter = warp & 3;
+            const int epart = e >> 2;
+            const int row = quarter * 32 + lane;
             const int tile = blockIdx.x;
             const int m0 = (tile / p.n_tiles) * BT;
-            const int n = (tile % p.n_tiles) * kBlockN + row;
-            const uint32_t rank = cluster_ctarank();
+            const int n = (tile % p.n_tiles) * p.rows + row;
+            const int rank = static_cast<int>(cluster_ctarank());
+            const int per_rank = ((BT + p.ksplit - 1) / p.ksplit + 3) / 4 * 4;
+            const int cb = rank * per_rank;
+            const int ce = min(BT, cb + per_rank);
             const uint32_t part0 = smem_u32(smem);
-            if (n < p.N) {
-                for (int c = static_cast<int>(rank); c < BT; c += p.ksplit) {
-                    const int m = m0 + c;
-                    if (m >= p.M) break;
-                    const uint32_t off = static_cast<uint32_t>((c * kBlockN + row) * 4);
-                    float acc = 0.f;
-                    for (int q = 0; q < p.ksplit; ++q) acc += ld_shared_cluster_f32(map_shared_rank(part0 + off, q));
-                    p.Y[static_cast<size_t>(m) * p.N + n] = __float2bfloat16_rn(acc * p.rowmul[m]);
+            if (row < p.rows && n < p.N) {
+                for (int c = cb + 4 * epart; c < ce; c += 4 * C::kEpiParts) {
+                    if (m0 + c >= p.M) break;
+                    const int pc = (c >> 2) ^ (row & C::kPartSwizzle);
+                    const uint32_t off = static_cast<uint32_t>((row * BT + pc * 4) * 4);
+                    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                    for (int q = 0; q < p.ksplit; ++q) {
+                        const float4 v = ld_shared_cluster_v4(map_shared_rank(part0 + off, q));
+                        acc.x += v.x;
+                        acc.y += v.y;
+                        acc.z += v.z;
+                        acc.w += v.w;
+                    }
+                    const float a4[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int m = m0 + c + j;
+                        if (m < p.M)
+                            p.Y[static_cast<size_t>(m) * p.N + n] = __float2bfloat16_rn(a4[j] * p.rowmul[m]);
+                    }
                 }
             }
         }
@@ -591,7 +699,7 @@ int num_sms() {
 }
 
 template <int BITS, int GS, int BT>
-lowbit_status launch(const GemmProblem& g, int ksplit_request, cudaStream_t stream) {
+lowbit_status launch(const GemmProblem& g, int rows, int ksplit_request, cudaStream_t stream) {
     using C = Cfg<BITS, GS, BT>;
     auto kernel = lowbit_gemm_kernel<BITS, GS, BT>;
     static bool attr_done = false;
@@ -611,7 +719,7 @@ lowbit_status launch(const GemmProblem& g, int ksplit_request, cudaStream_t stre
     bool ok = make_map_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, xh, K, M, uint64_t(K) * 2, 64, BT,
                           CU_TENSOR_MAP_SWIZZLE_128B);
     ok = ok && make_map_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, g.Wp, uint64_t(K) * BITS / 32, N,
-                           uint64_t(K) * BITS / 8, C::kWordsPerRow, kBlockN, wswz);
+                           uint64_t(K) * BITS / 8, C::kWordsPerRow, rows, wswz);
     ok = ok && make_map_2d(&ms, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, g.scales, N, K / GS, uint64_t(N) * 2, kBlockN,
                            C::kGroupsPerStage, CU_TENSOR_MAP_SWIZZLE_NONE);
     if (BITS == 4)
@@ -626,8 +734,10 @@ lowbit_status launch(const GemmProblem& g, int ksplit_request, cudaStream_t stre
     p.N = N;
     p.K = K;
     p.num_kb = (K + kBlockK - 1) / kBlockK;
+    p.rows = rows;
+    p.tx_bytes = static_cast<uint32_t>(C::kTxFixed + rows * C::kWRowBytes);
     p.m_tiles = (M + BT - 1) / BT;
-    p.n_tiles = (N + kBlockN - 1) / kBlockN;
+    p.n_tiles = (N + rows - 1) / rows;
     p.num_tiles = p.m_tiles * p.n_tiles;
     p.Y = static_cast<__nv_bfloat16*>(g.Y);
     p.rowmul = rowmul;
@@ -695,43 +805,59 @@ int pick_bt(int64_t M) {
 int ctas_per_sm_for(int bt) { return bt <= 64 ? 2 : 1; }
 
 template <int BITS, int GS>
-lowbit_status launch_bits_gs(const GemmProblem& g, int bt, int ksplit, cudaStream_t s) {
+lowbit_status launch_bits_gs(const GemmProblem& g, int bt, int rows, int ksplit, cudaStream_t s) {
     switch (bt) {
-        case 16: return launch<BITS, GS, 16>(g, ksplit, s);
-        case 32: return launch<BITS, GS, 32>(g, ksplit, s);
-        case 64: return launch<BITS, GS, 64>(g, ksplit, s);
-        case 128: return launch<BITS, GS, 128>(g, ksplit, s);
-        case 256: return launch<BITS, GS, 256>(g, ksplit, s);
+        case 16: return launch<BITS, GS, 16>(g, rows, ksplit, s);
+        case 32: return launch<BITS, GS, 32>(g, rows, ksplit, s);
+        case 64: return launch<BITS, GS, 64>(g, rows, ksplit, s);
+        case 128: return launch<BITS, GS, 128>(g, rows, ksplit, s);
+        case 256: return launch<BITS, GS, 256>(g, rows, ksplit, s);
         default: return LOWBIT_ERR_UNSUPPORTED;
     }
 }
 
 }  // namespace
 
-// Chooses the tile width and split-K factor, then launches. `force_bt` / `force_split`
-// (0 = automatic) pin them for tests and tuning.
-lowbit_status gemm_launch(const GemmProblem& g, int force_bt, int force_split, cudaStream_t stream) {
+// Chooses the launch configuration (tile_tokens, tile_rows, ksplit), each 0 = automatic:
+//   * one token tile and small M (weight streaming, HBM-bound): either "flat" tiles of
+//     ceil(N / #SMs) rows (a multiple of 8) with the whole K per CTA and no reduction, or 128-row
+//     tiles with K split over a cluster, whichever reads fewer X bytes per weight byte;
+//   * few tiles otherwise: 128-row tiles with K split over a cluster;
+//   * many tiles: 128-row tiles on a persistent grid.
+lowbit_status gemm_launch(const GemmProblem& g, int force_bt, int force_rows, int force_split,
+                          cudaStream_t stream) {
     const int bt = force_bt ? force_bt : pick_bt(g.M);
+    const int sms = num_sms();
+    const int64_t num_kb = (g.K + kBlockK - 1) / kBlockK;
+    const int64_t m_tiles = (g.M + bt - 1) / bt;
+    int rows = force_rows ? force_rows : kBlockN;
     int ksplit = force_split;
-    if (!ksplit) {
-        const int64_t tiles = ((g.M + bt - 1) / bt) * ((g.N + kBlockN - 1) / kBlockN);
-        const int64_t slots = static_cast<int64_t>(num_sms()) * ctas_per_sm_for(bt);
-        const int64_t num_kb = (g.K + kBlockK - 1) / kBlockK;
+    if (!force_rows && !force_split) {
+        const int64_t slots = static_cast<int64_t>(sms) * ctas_per_sm_for(bt);
+        const int64_t tiles128 = m_tiles * ((g.N + kBlockN - 1) / kBlockN);
+        int64_t flat_rows = ((g.N + sms - 1) / sms + 7) / 8 * 8;
+        // X bytes read per packed-weight byte by one CTA: 2 * bt / (rows * bits / 8)
+        const double x_per_w = (2.0 * bt) / (static_cast<double>(flat_rows) * g.bits / 8.0);
         ksplit = 1;
-        if (tiles * 2 <= slots && num_kb >= 4) {
-            int64_t s = slots / tiles;
+        if (bt <= 64 && m_tiles == 1 && flat_rows < kBlockN && x_per_w <= 1.25) {
+            rows = static_cast<int>(flat_rows);
+        } else if (tiles128 * 2 <= slots && num_kb >= 4) {
+            const int64_t target = (bt <= 64 && m_tiles == 1) ? sms : slots;   // small M: one CTA per SM
+            int64_t s = target / tiles128;
             if (s > 8) s = 8;
             if (s > num_kb / 2) s = num_kb / 2;
             ksplit = static_cast<int>(s < 1 ? 1 : s);
         }
     }
+    if (!ksplit) ksplit = 1;
+    if (rows < 8 || rows > kBlockN || rows % 8) return LOWBIT_ERR_UNSUPPORTED;
     switch (g.bits * 1000 + g.group_size) {
-        case 1064: return launch_bits_gs<1, 64>(g, bt, ksplit, stream);
-        case 1128: return launch_bits_gs<1, 128>(g, bt, ksplit, stream);
-        case 2064: return launch_bits_gs<2, 64>(g, bt, ksplit, stream);
-        case 2128: return launch_bits_gs<2, 128>(g, bt, ksplit, stream);
-        case 4064: return launch_bits_gs<4, 64>(g, bt, ksplit, stream);
-        case 4128: return launch_bits_gs<4, 128>(g, bt, ksplit, stream);
+        case 1064: return launch_bits_gs<1, 64>(g, bt, rows, ksplit, stream);
+        case 1128: return launch_bits_gs<1, 128>(g, bt, rows, ksplit, stream);
+        case 2064: return launch_bits_gs<2, 64>(g, bt, rows, ksplit, stream);
+        case 2128: return launch_bits_gs<2, 128>(g, bt, rows, ksplit, stream);
+        case 4064: return launch_bits_gs<4, 64>(g, bt, rows, ksplit, stream);
+        case 4128: return launch_bits_gs<4, 128>(g, bt, rows, ksplit, stream);
         default: return LOWBIT_ERR_UNSUPPORTED;
     }
 }

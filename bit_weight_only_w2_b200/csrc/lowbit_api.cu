@@ -145,13 +145,13 @@ LOWBIT_API lowbit_status lowbit_gemm(int64_t M, int64_t N, int64_t K, int bits, 
     lowbit_status st = validate_gemm(g);
     if (st != LOWBIT_OK || M == 0 || N == 0) return st;
     if ((st = check_device()) != LOWBIT_OK) return st;
-    return gemm_launch(g, 0, 0, static_cast<cudaStream_t>(stream));
+    return gemm_launch(g, 0, 0, 0, static_cast<cudaStream_t>(stream));
 }
 
 LOWBIT_API lowbit_status lowbit_gemm_ex(int64_t M, int64_t N, int64_t K, int bits, int group_size, const void* X,
                                         const uint32_t* Wp, const void* scales, const void* zeros, void* Y,
-                                        void* workspace, size_t workspace_bytes, int tile_tokens, int ksplit,
-                                        void* stream) {
+                                        void* workspace, size_t workspace_bytes, int tile_tokens, int tile_rows,
+                                        int ksplit, void* stream) {
     const GemmProblem g = make_problem(M, N, K, bits, group_size, X, Wp, scales, zeros, Y, workspace, workspace_bytes);
     lowbit_status st = validate_gemm(g);
     if (st != LOWBIT_OK || M == 0 || N == 0) return st;
@@ -159,8 +159,9 @@ LOWBIT_API lowbit_status lowbit_gemm_ex(int64_t M, int64_t N, int64_t K, int bit
         tile_tokens != 256)
         return LOWBIT_ERR_UNSUPPORTED;
     if (ksplit < 0 || ksplit > 8) return LOWBIT_ERR_UNSUPPORTED;
+    if (tile_rows < 0 || tile_rows > 128 || tile_rows % 8 != 0) return LOWBIT_ERR_UNSUPPORTED;
     if ((st = check_device()) != LOWBIT_OK) return st;
-    return gemm_launch(g, tile_tokens, ksplit, static_cast<cudaStream_t>(stream));
+    return gemm_launch(g, tile_tokens, tile_rows, ksplit, static_cast<cudaStream_t>(stream));
 }
 
 LOWBIT_API lowbit_status lowbit_gemm_batch(const lowbit_gemm_desc* descs, int count, void* workspace,
@@ -180,7 +181,7 @@ LOWBIT_API lowbit_status lowbit_gemm_batch(const lowbit_gemm_desc* descs, int co
         if (d.M == 0 || d.N == 0) continue;
         st = gemm_launch(make_problem(d.M, d.N, d.K, d.bits, d.group_size, d.X, d.Wp, d.scales, d.zeros, d.Y,
                                       workspace, workspace_bytes),
-                         0, 0, static_cast<cudaStream_t>(stream));
+                         0, 0, 0, static_cast<cudaStream_t>(stream));
         if (st != LOWBIT_OK) return st;
     }
     return LOWBIT_OK;

@@ -35,8 +35,10 @@ inline WorkspaceLayout workspace_layout(int64_t M, int64_t K) {
 // Validates one problem against the ABI's preconditions (no launch, no CUDA call).
 lowbit_status validate_gemm(const GemmProblem& g);
 
-// Launches the GEMM kernel for a validated problem. force_bt / force_split: 0 = automatic.
-lowbit_status gemm_launch(const GemmProblem& g, int force_bt, int force_split, cudaStream_t stream);
+// Launches the X conversion and the GEMM kernel for a validated problem. force_bt (tokens per
+// tile), force_rows (weight rows per tile) and force_split (K slices): 0 = automatic.
+lowbit_status gemm_launch(const GemmProblem& g, int force_bt, int force_rows, int force_split,
+                          cudaStream_t stream);
 
 // Reads (and optionally clears) the device status word. Synchronises the device.
 lowbit_status read_device_status(int clear);

@@ -108,14 +108,17 @@ lowbit_status lowbit_gemm(int64_t M, int64_t N, int64_t K, int bits, int group_s
                           void* workspace, size_t workspace_bytes, void* stream);
 
 /* lowbit_gemm with the kernel configuration fixed instead of chosen from the shape, for
- * tuning and tests: `tile_tokens` = tokens per CTA tile (16, 32, 64, 128 or 256; 0 = automatic),
- * `ksplit` = number of K slices summed across a thread-block cluster (1..8; 0 = automatic,
- * 1 = no split). Other arguments and all checks are those of lowbit_gemm; an unsupported
- * tile_tokens returns LOWBIT_ERR_UNSUPPORTED. */
+ * tuning and tests (each 0 = automatic):
+ *   tile_tokens  tokens per CTA tile: 16, 32, 64, 128 or 256
+ *   tile_rows    weight rows per CTA tile: a multiple of 8 up to 128 (128 unless the shape is
+ *                small; fewer rows give more CTAs, each streaming the whole K)
+ *   ksplit       number of K slices summed across a thread-block cluster, 1..8 (1 = no split)
+ * Other arguments and all checks are those of lowbit_gemm; values outside these sets return
+ * LOWBIT_ERR_UNSUPPORTED. */
 lowbit_status lowbit_gemm_ex(int64_t M, int64_t N, int64_t K, int bits, int group_size, const void* X,
                              const uint32_t* Wp, const void* scales, const void* zeros, void* Y,
-                             void* workspace, size_t workspace_bytes, int tile_tokens, int ksplit,
-                             void* stream);
+                             void* workspace, size_t workspace_bytes, int tile_tokens, int tile_rows,
+                             int ksplit, void* stream);
 
 /* One linear of a chain, with the meaning and layout of lowbit_gemm's arguments. */
 typedef struct lowbit_gemm_desc {

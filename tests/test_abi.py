@@ -86,9 +86,13 @@ def test_gemm_rejects_before_launch(lib, args, expect):
 
 
 def test_gemm_ex_rejects_bad_tile(lib):
-    st = lib.lowbit_gemm_ex(16, 128, 256, 2, 128, A, A, A, None, A, A, WS, 48, 0, None)
+    st = lib.lowbit_gemm_ex(16, 128, 256, 2, 128, A, A, A, None, A, A, WS, 48, 0, 0, None)
     assert st == 3
-    st = lib.lowbit_gemm_ex(16, 128, 256, 2, 128, A, A, A, None, A, A, WS, 16, 9, None)
+    st = lib.lowbit_gemm_ex(16, 128, 256, 2, 128, A, A, A, None, A, A, WS, 16, 0, 9, None)
+    assert st == 3
+    st = lib.lowbit_gemm_ex(16, 128, 256, 2, 128, A, A, A, None, A, A, WS, 16, 20, 0, None)   # rows % 8
+    assert st == 3
+    st = lib.lowbit_gemm_ex(16, 128, 256, 2, 128, A, A, A, None, A, A, WS, 16, 136, 0, None)  # rows > 128
     assert st == 3
 
 

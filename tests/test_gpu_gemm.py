@@ -57,7 +57,7 @@ _ref_cache = {}
 
 @pytest.mark.parametrize("bits,gs", FORMATS)
 @pytest.mark.parametrize("tile_tokens", [16, 32, 64, 128, 256])
-@pytest.mark.parametrize("ksplit", [1, 2, 3])
+@pytest.mark.parametrize("ksplit", [1, 2, 3, 7])
 def test_gemm_every_tile_config(bits, gs, tile_tokens, ksplit):
     spec = spec_for(bits, gs, 200, 768, 264, seed=7)
     key = (bits, gs)
@@ -67,6 +67,28 @@ def test_gemm_every_tile_config(bits, gs, tile_tokens, ksplit):
         _ref_cache[key] = (prob, ref)
     prob, ref = _ref_cache[key]
     run_and_compare(spec, tile_tokens, ksplit, prob=prob, ref=ref)
+
+
+_flat_cache = {}
+
+
+@pytest.mark.parametrize("bits,gs", FORMATS)
+@pytest.mark.parametrize("tile_tokens", [16, 32, 64])
+@pytest.mark.parametrize("tile_rows", [8, 40, 72, 120])
+def test_gemm_flat_row_tiles(bits, gs, tile_tokens, tile_rows):
+    """Small-M "flat" tiles: fewer than 128 weight rows per CTA, whole K per CTA, ragged N."""
+    spec = spec_for(bits, gs, 40, 768, 264, seed=9)
+    key = (bits, gs)
+    if key not in _flat_cache:
+        prob = synth.make_problem(spec)
+        ref = oracle.gemm(prob.x_bf16, _gpu.oracle_packed(prob), prob.scales, prob.zeros, spec.N, bits, gs)
+        _flat_cache[key] = (prob, ref)
+    prob, ref = _flat_cache[key]
+    x, packed, s, z = _gpu.dev_problem(prob)
+    y = lb.gemm(x, packed, s, z, bits, gs, tile_tokens=tile_tokens, tile_rows=tile_rows, ksplit=1)
+    torch.cuda.synchronize()
+    assert lb.device_status() == 0
+    _gpu.check_close(_gpu.y_to_f64(y), ref, what=f"flat rows={tile_rows} bt={tile_tokens}")
 
 
 @pytest.mark.parametrize("bits,gs", [(2, 64), (4, 64)])
