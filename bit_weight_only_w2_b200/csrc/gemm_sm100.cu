@@ -93,26 +93,34 @@ struct Cfg {
     static constexpr int kGroupsPerStage = kBlockK / GS;            // 1 or 2
     static constexpr int kSBytes = kGroupsPerStage * kBlockN * 2;
     static constexpr int kZBytes = (BITS == 4) ? kSBytes : 0;
-    static constexpr int kXOff = 0;
-    static constexpr int kWOff = kXBytes;
-    static constexpr int kSOff = kWOff + kWBytes;
+    // Two rings in shared memory: X stages (the MMA's B operand, freed by the MMA) and weight
+    // stages (packed codes + scales + zeros, freed by the dequant warps). The weight ring runs
+    // ahead of the X ring, so decoding never waits for X. One X stage is one 128-wide k-block,
+    // fetched by a single TMA request (large requests stream from L2 faster than small ones).
+    static constexpr int kXStageBytes = kXBytes;                    // a multiple of 2048
+    static constexpr int kWOff = 0;
+    static constexpr int kSOff = kWBytes;
     static constexpr int kZOff = kSOff + kSBytes;
-    static constexpr int kStageBytes = (kZOff + kZBytes + 1023) / 1024 * 1024;
-    static constexpr int kTxFixed = kXBytes + kSBytes + kZBytes;   // plus rows * kWRowBytes
+    static constexpr int kWStageBytes = (kZOff + kZBytes + 1023) / 1024 * 1024;
+    static constexpr int kWTxFixed = kSBytes + kZBytes;            // plus rows * kWRowBytes
     static constexpr int kBarBytes = 1024;
     static constexpr int kBudget = kSmemLimit / kCtasPerSm - 1024 /*align*/ - kBarBytes - 2048 /*reserve*/;
-    static constexpr int kStagesFit = kBudget / kStageBytes;
-    static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
-    static_assert(kStages >= 2, "shared memory");
+    static constexpr int kXStagesFit = (kBudget - 2 * kWStageBytes) / kXStageBytes;
+    static constexpr int kXStages = kXStagesFit > 8 ? 8 : kXStagesFit;
+    static constexpr int kWStagesFit = (kBudget - kXStages * kXStageBytes) / kWStageBytes;
+    static constexpr int kWStages = kWStagesFit > 8 ? 8 : kWStagesFit;
+    static_assert(kXStages >= 2 && kWStages >= 2, "shared memory");
+    static constexpr int kWRingOff = kXStages * kXStageBytes;
+    static constexpr int kBarOff = kWRingOff + kWStages * kWStageBytes;
     // Request enough shared memory that at most kCtasPerSm CTAs of these kernels share an SM:
     // tensor memory (512 columns per SM) is not a scheduling resource, so residency is capped
     // through shared memory instead (228 KB per SM).
-    static constexpr int kSmemNeeded = 1024 + kStages * kStageBytes + kBarBytes;
+    static constexpr int kSmemNeeded = 1024 + kBarOff + kBarBytes;
     static constexpr int kSmemFloor = (kCtasPerSm == 2) ? 80 * 1024 : 150 * 1024;
     static constexpr int kSmemBytes = kSmemNeeded > kSmemFloor ? kSmemNeeded : kSmemFloor;
     static_assert(kSmemBytes <= kSmemLimit, "shared memory");
-    // split-K partial tile (fp32 [128][BT], rows of 16-byte chunks XOR-swizzled) reuses the ring
-    static_assert(BT * kBlockN * 4 <= kStages * kStageBytes, "split-K partial buffer");
+    // split-K partial tile (fp32 [128][BT], rows of 16-byte chunks XOR-swizzled) reuses the X ring
+    static_assert(BT * kBlockN * 4 <= kXStages * kXStageBytes, "split-K partial buffer");
     static constexpr int kPartSwizzle = (BT / 4 >= 8) ? 7 : (BT / 4 - 1);
     static constexpr uint32_t kIdesc = idesc_f16_f32(kBlockN, BT);
 };
@@ -124,7 +132,7 @@ struct KernelParams {
     int rows;            // weight rows per tile: 128, or fewer (multiple of 8) for small M
     int m_tiles, n_tiles, num_tiles;
     int ksplit;          // cluster size along z (1 = no split)
-    uint32_t tx_bytes;   // bytes delivered into one pipeline stage
+    uint32_t wtx_bytes;  // bytes delivered into one weight stage
     __nv_bfloat16* Y;
     const float* rowmul; // per-row power-of-two factor written by the X conversion pass
 };
@@ -188,16 +196,19 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT>::kThreads, Cfg<BITS, GS, BT>
                        const __grid_constant__ CUtensorMap map_s, const __grid_constant__ CUtensorMap map_z,
                        const KernelParams p) {
     using C = Cfg<BITS, GS, BT>;
-    constexpr int S = C::kStages;
+    constexpr int SX = C::kXStages;
+    constexpr int SW = C::kWStages;
     constexpr int NA = C::kNumA;
     constexpr int NACC = C::kNumAcc;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* bar_area = smem + S * C::kStageBytes;
-    uint64_t* full = reinterpret_cast<uint64_t*>(bar_area);
-    uint64_t* empty = full + S;
-    uint64_t* afull = empty + S;
+    uint8_t* wring = smem + C::kWRingOff;
+    uint64_t* xfull = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+    uint64_t* xempty = xfull + SX;
+    uint64_t* wfull = xempty + SX;
+    uint64_t* wempty = wfull + SW;
+    uint64_t* afull = wempty + SW;
     uint64_t* aempty = afull + NA;
     uint64_t* accfull = aempty + NA;
     uint64_t* accempty = accfull + NACC;
@@ -209,9 +220,13 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT>::kThreads, Cfg<BITS, GS, BT>
     const int lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < S; ++i) {
-            mbar_init(&full[i], 1);
-            mbar_init(&empty[i], 1 + C::kNumDqWarps);
+        for (int i = 0; i < SX; ++i) {
+            mbar_init(&xfull[i], 1);
+            mbar_init(&xempty[i], 1);
+        }
+        for (int i = 0; i < SW; ++i) {
+            mbar_init(&wfull[i], 1);
+            mbar_init(&wempty[i], C::kNumDqWarps);
         }
         for (int i = 0; i < NA; ++i) {
             mbar_init(&afull[i], C::kNumDqWarps);
@@ -263,48 +278,69 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT>::kThreads, Cfg<BITS, GS, BT>
                 m0 = (tile / p.n_tiles) * BT;
                 n0 = (tile % p.n_tiles) * p.rows;
             };
-            auto load_weights = [&](uint32_t it) {
+            auto issue_w = [&](uint32_t it) {
                 int m0, n0, kb;
                 coords(it, m0, n0, kb);
-                const uint32_t s = it % S;
-                uint8_t* st = smem + s * C::kStageBytes;
-                mbar_arrive_expect_tx(&full[s], p.tx_bytes);
-                tma_load_2d(&map_w, &full[s], st + C::kWOff, kb * C::kWordsPerRow, n0);
-                tma_load_2d(&map_s, &full[s], st + C::kSOff, n0, kb * C::kGroupsPerStage);
-                if (BITS == 4) tma_load_2d(&map_z, &full[s], st + C::kZOff, n0, kb * C::kGroupsPerStage);
+                const uint32_t s = it % SW;
+                uint8_t* st = wring + s * C::kWStageBytes;
+                mbar_arrive_expect_tx(&wfull[s], p.wtx_bytes);
+                tma_load_2d(&map_w, &wfull[s], st + C::kWOff, kb * C::kWordsPerRow, n0);
+                tma_load_2d(&map_s, &wfull[s], st + C::kSOff, n0, kb * C::kGroupsPerStage);
+                if (BITS == 4) tma_load_2d(&map_z, &wfull[s], st + C::kZOff, n0, kb * C::kGroupsPerStage);
             };
-            auto load_x = [&](uint32_t it) {
+            auto issue_x = [&](uint32_t it) {
                 int m0, n0, kb;
                 coords(it, m0, n0, kb);
-                const uint32_t s = it % S;
-                uint8_t* st = smem + s * C::kStageBytes;
-                tma_load_2d(&map_x, &full[s], st + C::kXOff, kb * kBlockK, m0);
-                tma_load_2d(&map_x, &full[s], st + C::kXOff + C::kXHalfBytes, kb * kBlockK + 64, m0);
+                const uint32_t s = it % SX;
+                uint8_t* st = smem + s * C::kXStageBytes;
+                mbar_arrive_expect_tx(&xfull[s], C::kXBytes);
+                // box (64 k, BT tokens, 2 halves) = both 128-byte-swizzled K halves in one request
+                tma_load_3d(&map_x, &xfull[s], st, 0, m0, kb * 2);
             };
             // The packed weights and scales are not written by the kernel just before this one
             // (the X conversion, which itself starts only once everything earlier in the stream
-            // has completed), so the first stages' weight boxes are requested before waiting for
-            // it; their X boxes follow as soon as the conversion is done.
-            const uint32_t pre = total < static_cast<uint32_t>(S) ? total : static_cast<uint32_t>(S);
-            for (uint32_t it = 0; it < pre; ++it) load_weights(it);
+            // has completed), so the first weight stages are requested before waiting for it.
+            uint32_t itw = 0, itx = 0;
+            const uint32_t wpre = total < static_cast<uint32_t>(SW) ? total : static_cast<uint32_t>(SW);
+            for (; itw < wpre; ++itw) issue_w(itw);
             grid_dependency_wait();
-            for (uint32_t it = 0; it < pre; ++it) load_x(it);
-            uint32_t it = pre;
+            // Fill both rings as their slots free up, without blocking on either.
             bool ok = true;
-            for (; it < total; ++it) {
-                const uint32_t s = it % S, ph = (it / S) & 1u;
-                if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, status)) {
-                    ok = false;
-                    break;
+            long long t_last = clock64();
+            uint32_t idle = 0;
+            while (itx < total || itw < total) {
+                bool progress = false;
+                if (itx < total && mbar_test_wait(&xempty[itx % SX], ((itx / SX) & 1u) ^ 1u)) {
+                    issue_x(itx++);
+                    progress = true;
                 }
-                load_weights(it);
-                load_x(it);
+                if (itw < total && mbar_test_wait(&wempty[itw % SW], ((itw / SW) & 1u) ^ 1u)) {
+                    issue_w(itw++);
+                    progress = true;
+                }
+                if (progress) {
+                    idle = 0;
+                    t_last = clock64();
+                } else if ((++idle & 63u) == 0) {
+                    if (*abort_flag) { ok = false; break; }
+                    if (clock64() - t_last > kWaitLimitCycles) {
+                        atomicOr(status, kDevErrTimeout);
+                        *abort_flag = 1;
+                        ok = false;
+                        break;
+                    }
+                }
             }
             if (!ok) {
                 // Drain: wait (bounded) for the copies still in flight before the CTA exits.
-                for (uint32_t j = (it > static_cast<uint32_t>(S) ? it - S : 0u); j < it; ++j) {
+                for (uint32_t j = (itx > static_cast<uint32_t>(SX) ? itx - SX : 0u); j < itx; ++j) {
                     const long long t0 = clock64();
-                    while (!mbar_try_wait(&full[j % S], (j / S) & 1u) && clock64() - t0 < kWaitLimitCycles) {
+                    while (!mbar_try_wait(&xfull[j % SX], (j / SX) & 1u) && clock64() - t0 < kWaitLimitCycles) {
+                    }
+                }
+                for (uint32_t j = (itw > static_cast<uint32_t>(SW) ? itw - SW : 0u); j < itw; ++j) {
+                    const long long t0 = clock64();
+                    while (!mbar_try_wait(&wfull[j % SW], (j / SW) & 1u) && clock64() - t0 < kWaitLimitCycles) {
                     }
                 }
             }
@@ -324,12 +360,12 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT>::kThreads, Cfg<BITS, GS, BT>
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + b * BT;
                 for (int kb = kb_begin; kb < kb_end; ++kb, ++it, ++ait) {
-                    const uint32_t s = it % S, ph = (it / S) & 1u;
+                    const uint32_t s = it % SX, ph = (it / SX) & 1u;
                     const uint32_t a = ait % NA, aph = (ait / NA) & 1u;
-                    if (!mbar_wait(&full[s], ph, abort_flag, status)) { ok = false; break; }
+                    if (!mbar_wait(&xfull[s], ph, abort_flag, status)) { ok = false; break; }
                     if (!mbar_wait(&afull[a], aph, abort_flag, status)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t xs = smem_u32(smem + s * C::kStageBytes + C::kXOff);
+                    const uint32_t xs = smem_u32(smem + s * C::kXStageBytes);
 #pragma unroll
                     for (int kk = 0; kk < kBlockK / 16; ++kk) {
                         const uint32_t a_tmem = tmem_base + C::kACol0 + a * 64 + kk * 8;
@@ -338,7 +374,7 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT>::kThreads, Cfg<BITS, GS, BT>
                         mma_f16_ts(d_tmem, a_tmem, bdesc, C::kIdesc, (kb > kb_begin || kk > 0) ? 1u : 0u);
                     }
                     issued = true;
-                    mma_commit(&empty[s]);
+                    mma_commit(&xempty[s]);
                     mma_commit(&aempty[a]);
                 }
                 if (!ok) break;
@@ -365,10 +401,10 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT>::kThreads, Cfg<BITS, GS, BT>
         bool ok = true;
         for (int t = 0; t < my_tiles && ok; ++t) {
             for (int kb = kb_begin; kb < kb_end; ++kb, ++it, ++ait) {
-                const uint32_t s = it % S, ph = (it / S) & 1u;
+                const uint32_t s = it % SW, ph = (it / SW) & 1u;
                 const uint32_t a = ait % NA, aph = (ait / NA) & 1u;
-                if (!__all_sync(0xffffffffu, mbar_wait(&full[s], ph, abort_flag, status))) { ok = false; break; }
-                const uint8_t* st = smem + s * C::kStageBytes;
+                if (!__all_sync(0xffffffffu, mbar_wait(&wfull[s], ph, abort_flag, status))) { ok = false; break; }
+                const uint8_t* st = wring + s * C::kWStageBytes;
                 // --- this row's packed words and scales (rows past the tile decode to zero)
                 uint32_t words[kHalvesPerPart][C::kWordsPerRow / 2];
                 uint32_t s2[kHalvesPerPart], c2[kHalvesPerPart];
@@ -412,7 +448,7 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT>::kThreads, Cfg<BITS, GS, BT>
                     }
                 }
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[s]);
+                if (lane == 0) mbar_arrive(&wempty[s]);
                 // --- decode into the tensor-memory A ring
                 if (!__all_sync(0xffffffffu, mbar_wait(&aempty[a], aph ^ 1u, abort_flag, status))) {
                     ok = false;
@@ -672,6 +708,21 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
     return fn;
 }
 
+// X as a 3-D tensor (64 k, M rows, K/64 k-atoms) so that one box covers a whole 128-wide k-block
+// of BT token rows in the 128-byte-swizzled layout [k half][row][64 k] the MMA reads.
+bool make_map_x3d(CUtensorMap* map, const void* base, uint64_t M, uint64_t K, uint32_t box_rows) {
+    auto fn = get_encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {64, M, K / 64};
+    cuuint64_t strides[2] = {K * 2, 128};
+    cuuint32_t box[3] = {64, box_rows, 2};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 bool make_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, int elem_bytes, const void* base, uint64_t inner,
                  uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
                  CUtensorMapSwizzle swz) {
@@ -716,8 +767,7 @@ lowbit_status launch(const GemmProblem& g, int rows, int ksplit_request, cudaStr
     const WorkspaceLayout ws = workspace_layout(g.M, g.K);
     void* xh = g.workspace;
     float* rowmul = reinterpret_cast<float*>(static_cast<uint8_t*>(g.workspace) + ws.rowmul_offset);
-    bool ok = make_map_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, xh, K, M, uint64_t(K) * 2, 64, BT,
-                          CU_TENSOR_MAP_SWIZZLE_128B);
+    bool ok = make_map_x3d(&mx, xh, M, K, BT);
     ok = ok && make_map_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, g.Wp, uint64_t(K) * BITS / 32, N,
                            uint64_t(K) * BITS / 8, C::kWordsPerRow, rows, wswz);
     ok = ok && make_map_2d(&ms, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, g.scales, N, K / GS, uint64_t(N) * 2, kBlockN,
@@ -735,7 +785,7 @@ lowbit_status launch(const GemmProblem& g, int rows, int ksplit_request, cudaStr
     p.K = K;
     p.num_kb = (K + kBlockK - 1) / kBlockK;
     p.rows = rows;
-    p.tx_bytes = static_cast<uint32_t>(C::kTxFixed + rows * C::kWRowBytes);
+    p.wtx_bytes = static_cast<uint32_t>(C::kWTxFixed + rows * C::kWRowBytes);
     p.m_tiles = (M + BT - 1) / BT;
     p.n_tiles = (N + rows - 1) / rows;
     p.num_tiles = p.m_tiles * p.n_tiles;
