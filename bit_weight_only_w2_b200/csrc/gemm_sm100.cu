@@ -670,6 +670,24 @@ __global__ void __launch_bounds__(kConvThreads) convert_x_kernel(const uint4* __
     if (threadIdx.x == 0) rowmul[row] = __int_as_float((127 + e) << 23);   // 2^e
 }
 
+lowbit_status launch_convert_x(const GemmProblem& g, cudaStream_t stream) {
+    const WorkspaceLayout ws = workspace_layout(g.M, g.K);
+    cudaLaunchConfig_t ccfg = {};
+    cudaLaunchAttribute cattr[1];
+    cattr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    cattr[0].val.programmaticStreamSerializationAllowed = 1;
+    ccfg.gridDim = dim3(static_cast<unsigned>(g.M), 1, 1);
+    ccfg.blockDim = dim3(kConvThreads, 1, 1);
+    ccfg.stream = stream;
+    ccfg.attrs = cattr;
+    ccfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(
+        &ccfg, convert_x_kernel, static_cast<const uint4*>(g.X), static_cast<int>(g.K / 8),
+        static_cast<uint4*>(g.workspace),
+        reinterpret_cast<float*>(static_cast<uint8_t*>(g.workspace) + ws.rowmul_offset));
+    return e == cudaSuccess ? LOWBIT_OK : LOWBIT_ERR_CUDA;
+}
+
 // One CTA waits on a barrier that nothing arrives on, with the GEMM's bounded wait: the wait
 // gives up after `limit` clocks and records the timeout in the device status word.
 __global__ void bounded_wait_selftest_kernel(long long limit) {
@@ -723,6 +741,8 @@ bool make_map_x3d(CUtensorMap* map, const void* base, uint64_t M, uint64_t K, ui
     return r == CUDA_SUCCESS;
 }
 
+}  // namespace
+
 bool make_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, int elem_bytes, const void* base, uint64_t inner,
                  uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
                  CUtensorMapSwizzle swz) {
@@ -748,6 +768,8 @@ int num_sms() {
     }
     return sms;
 }
+
+namespace {
 
 template <int BITS, int GS, int BT>
 lowbit_status launch(const GemmProblem& g, int rows, int ksplit_request, cudaStream_t stream) {
@@ -802,20 +824,7 @@ lowbit_status launch(const GemmProblem& g, int rows, int ksplit_request, cudaStr
 
     // X -> fp16 copy in the workspace, then the GEMM; both launched as programmatic dependents
     // of whatever precedes them on the stream.
-    {
-        cudaLaunchConfig_t ccfg = {};
-        cudaLaunchAttribute cattr[1];
-        cattr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        cattr[0].val.programmaticStreamSerializationAllowed = 1;
-        ccfg.gridDim = dim3(M, 1, 1);
-        ccfg.blockDim = dim3(kConvThreads, 1, 1);
-        ccfg.stream = stream;
-        ccfg.attrs = cattr;
-        ccfg.numAttrs = 1;
-        if (cudaLaunchKernelEx(&ccfg, convert_x_kernel, static_cast<const uint4*>(g.X), K / 8,
-                               static_cast<uint4*>(xh), rowmul) != cudaSuccess)
-            return LOWBIT_ERR_CUDA;
-    }
+    if (launch_convert_x(g, stream) != LOWBIT_OK) return LOWBIT_ERR_CUDA;
 
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attrs[2];
@@ -876,6 +885,9 @@ lowbit_status launch_bits_gs(const GemmProblem& g, int bt, int rows, int ksplit,
 //   * many tiles: 128-row tiles on a persistent grid.
 lowbit_status gemm_launch(const GemmProblem& g, int force_bt, int force_rows, int force_split,
                           cudaStream_t stream) {
+    // tile_tokens == 1 selects the small-M warp-MMA kernel; automatic choice for M <= 16
+    if (force_bt == 1) return gemv_launch(g, force_split, stream);
+    if (!force_bt && !force_rows && !force_split && gemv_supported(g)) return gemv_launch(g, 0, stream);
     const int bt = force_bt ? force_bt : pick_bt(g.M);
     const int sms = num_sms();
     const int64_t num_kb = (g.K + kBlockK - 1) / kBlockK;
@@ -910,6 +922,19 @@ lowbit_status gemm_launch(const GemmProblem& g, int force_bt, int force_rows, in
         case 4128: return launch_bits_gs<4, 128>(g, bt, rows, ksplit, stream);
         default: return LOWBIT_ERR_UNSUPPORTED;
     }
+}
+
+unsigned* device_status_address() {
+    constexpr int kMaxDevices = 64;
+    static unsigned* ptrs[kMaxDevices] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    if (!ptrs[dev]) {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_device_status) != cudaSuccess) return nullptr;
+        ptrs[dev] = static_cast<unsigned*>(ptr);
+    }
+    return ptrs[dev];
 }
 
 lowbit_status read_device_status(int clear) {

@@ -1,6 +1,7 @@
 // Declarations shared by the library's translation units (host side).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -39,6 +40,24 @@ lowbit_status validate_gemm(const GemmProblem& g);
 // tile), force_rows (weight rows per tile) and force_split (K slices): 0 = automatic.
 lowbit_status gemm_launch(const GemmProblem& g, int force_bt, int force_rows, int force_split,
                           cudaStream_t stream);
+
+// Launches the X -> fp16 conversion pass into the problem's workspace (programmatic dependent
+// launch). The GEMM kernels read its output.
+lowbit_status launch_convert_x(const GemmProblem& g, cudaStream_t stream);
+
+// Small-M GEMM (M <= 16) on warp-level tensor-core MMAs: launches the X conversion, then the
+// kernel. ksplit: 0 = automatic. gemv_supported: whether the shape fits that kernel.
+bool gemv_supported(const GemmProblem& g);
+lowbit_status gemv_launch(const GemmProblem& g, int ksplit, cudaStream_t stream);
+
+// Device address of the current device's status word (nullptr on failure).
+unsigned* device_status_address();
+
+// 2-D tiled tensor map (inner dimension contiguous) and the device's SM count.
+bool make_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, int elem_bytes, const void* base, uint64_t inner,
+                 uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                 CUtensorMapSwizzle swz);
+int num_sms();
 
 // Reads (and optionally clears) the device status word. Synchronises the device.
 lowbit_status read_device_status(int clear);

@@ -91,6 +91,29 @@ def test_gemm_flat_row_tiles(bits, gs, tile_tokens, tile_rows):
     _gpu.check_close(_gpu.y_to_f64(y), ref, what=f"flat rows={tile_rows} bt={tile_tokens}")
 
 
+@pytest.mark.parametrize("bits,gs", FORMATS)
+@pytest.mark.parametrize("M", [1, 5, 16])
+@pytest.mark.parametrize("K,N,ksplit", [(256, 520, 1), (192 * 4, 264, 3), (2560, 1032, 0), (9728, 256, 0)])
+def test_gemm_small_m_warp_mma(bits, gs, M, K, N, ksplit):
+    """The small-M kernel (warp-level MMAs, K split over a cluster), ragged N, partial k-blocks."""
+    if bits == 1 and K % 128:
+        pytest.skip("binary needs K % 128 == 0")
+    spec = spec_for(bits, gs, M, K, N, seed=M * 7 + K)
+    prob = synth.make_problem(spec)
+    ref = oracle.gemm(prob.x_bf16, _gpu.oracle_packed(prob), prob.scales, prob.zeros, N, bits, gs)
+    x, packed, s, z = _gpu.dev_problem(prob)
+    y = lb.gemm(x, packed, s, z, bits, gs, tile_tokens=1, ksplit=ksplit)
+    torch.cuda.synchronize()
+    assert lb.device_status() == 0
+    _gpu.check_close(_gpu.y_to_f64(y), ref, what=f"warp-mma M={M} K={K} N={N} split={ksplit}")
+
+
+def test_gemm_small_m_k_partial_block():
+    """K a multiple of 64 but not of 128 on the small-M kernel (last k-block half out of range)."""
+    spec = spec_for(2, 64, 9, 192, 136, seed=2)
+    run_and_compare(spec, tile_tokens=1)
+
+
 @pytest.mark.parametrize("bits,gs", [(2, 64), (4, 64)])
 def test_k_single_group_partial_stage(bits, gs):
     # K = 64: one half-filled stage of 128; the other half reads out of bounds (zero-filled)
