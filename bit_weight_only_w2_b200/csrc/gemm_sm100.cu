@@ -743,6 +743,19 @@ bool make_map_x3d(CUtensorMap* map, const void* base, uint64_t M, uint64_t K, ui
 
 }  // namespace
 
+bool make_map_3d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, const uint64_t (&dims)[3],
+                 const uint64_t (&strides)[2], const uint32_t (&box)[3], CUtensorMapSwizzle swz) {
+    auto fn = get_encode_fn();
+    if (!fn) return false;
+    cuuint64_t d[3] = {dims[0], dims[1], dims[2]};
+    cuuint64_t st[2] = {strides[0], strides[1]};
+    cuuint32_t b[3] = {box[0], box[1], box[2]};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, dtype, 3, const_cast<void*>(base), d, st, b, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 bool make_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, int elem_bytes, const void* base, uint64_t inner,
                  uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
                  CUtensorMapSwizzle swz) {
@@ -886,8 +899,8 @@ lowbit_status launch_bits_gs(const GemmProblem& g, int bt, int rows, int ksplit,
 lowbit_status gemm_launch(const GemmProblem& g, int force_bt, int force_rows, int force_split,
                           cudaStream_t stream) {
     // tile_tokens == 1 selects the small-M warp-MMA kernel; automatic choice for M <= 16
-    if (force_bt == 1) return gemv_launch(g, force_split, stream);
-    if (!force_bt && !force_rows && !force_split && gemv_supported(g)) return gemv_launch(g, 0, stream);
+    if (force_bt == 1) return smallm_launch(g, force_rows, force_split, stream);
+    if (!force_bt && !force_rows && !force_split && smallm_supported(g)) return smallm_launch(g, 0, 0, stream);
     const int bt = force_bt ? force_bt : pick_bt(g.M);
     const int sms = num_sms();
     const int64_t num_kb = (g.K + kBlockK - 1) / kBlockK;

@@ -158,7 +158,7 @@ LOWBIT_API lowbit_status lowbit_gemm_ex(int64_t M, int64_t N, int64_t K, int bit
     if (tile_tokens != 0 && tile_tokens != 1 && tile_tokens != 16 && tile_tokens != 32 && tile_tokens != 64 &&
         tile_tokens != 128 && tile_tokens != 256)
         return LOWBIT_ERR_UNSUPPORTED;
-    if (tile_tokens == 1 && (M > 16 || tile_rows != 0)) return LOWBIT_ERR_UNSUPPORTED;
+    if (tile_tokens == 1 && M > 16) return LOWBIT_ERR_UNSUPPORTED;
     if (ksplit < 0 || ksplit > 8) return LOWBIT_ERR_UNSUPPORTED;
     if (tile_rows < 0 || tile_rows > 128 || tile_rows % 8 != 0) return LOWBIT_ERR_UNSUPPORTED;
     if ((st = check_device()) != LOWBIT_OK) return st;

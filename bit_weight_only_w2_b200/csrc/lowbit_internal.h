@@ -45,10 +45,11 @@ lowbit_status gemm_launch(const GemmProblem& g, int force_bt, int force_rows, in
 // launch). The GEMM kernels read its output.
 lowbit_status launch_convert_x(const GemmProblem& g, cudaStream_t stream);
 
-// Small-M GEMM (M <= 16) on warp-level tensor-core MMAs: launches the X conversion, then the
-// kernel. ksplit: 0 = automatic. gemv_supported: whether the shape fits that kernel.
-bool gemv_supported(const GemmProblem& g);
-lowbit_status gemv_launch(const GemmProblem& g, int ksplit, cudaStream_t stream);
+// Small-M GEMM (M <= 16) on warp-level bf16 tensor-core MMAs, reading X directly (no
+// conversion pass, no workspace). rows (weight rows per CTA, multiple of 8, <= 128) and ksplit
+// (K slices per cluster, <= 8): 0 = automatic. smallm_supported: whether the shape fits it.
+bool smallm_supported(const GemmProblem& g);
+lowbit_status smallm_launch(const GemmProblem& g, int rows, int ksplit, cudaStream_t stream);
 
 // Device address of the current device's status word (nullptr on failure).
 unsigned* device_status_address();
@@ -58,6 +59,8 @@ bool make_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, int elem_bytes, co
                  uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
                  CUtensorMapSwizzle swz);
 int num_sms();
+bool make_map_3d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, const uint64_t (&dims)[3],
+                 const uint64_t (&strides)[2], const uint32_t (&box)[3], CUtensorMapSwizzle swz);
 
 // Reads (and optionally clears) the device status word. Synchronises the device.
 lowbit_status read_device_status(int clear);

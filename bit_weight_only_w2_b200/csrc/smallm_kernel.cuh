@@ -1,0 +1,556 @@
+// Small-M weight-only low-bit GEMM (M <= 16 tokens) for sm_100a: the HBM-bound case, e.g. the
+// Qwen3 text-encoder linears at 16 tokens (mlx-vlm Bonsai article, component architecture:
+// bits=4, group_size=64) or a GEMV-like decode step.
+//
+// At 16 tokens the work is streaming the packed weights; the multiply-accumulates still exceed
+// what CUDA-core FMAs sustain at HBM speed, so they run on warp-level tensor-core MMAs
+// (mma.sync m16n8k16, bf16 in, fp32 accumulate). tcgen05.mma is the wrong tool here: measured
+// on B200 it costs at least ~45 clocks per instruction with M = 128 however narrow N is, while
+// mma.sync sustains ~1000 MACs per clock per SM (one per ~8 clocks per SM sub-partition, also
+// with the decode instructions interleaved) and takes its B operand from registers, so decoded
+// weights need no staging. Its latency is long (~90 clocks when chains restart), so each warp
+// keeps up to eight independent accumulator chains (weight-row octets) in flight; the number
+// of octets per CTA is a template parameter so that a step's chains form one straight-line
+// block the compiler can interleave.
+//
+// Arithmetic. X is used as stored (bf16); codes are decoded WITHOUT their scale into exact bf16
+// values and the group scale is applied to fp32 group sums afterwards:
+//   binary   w = s * (+-1)                       -> decode +-1 exactly
+//   ternary  w = s * (f - 1),     f = t + 1       -> decode 128 + f exactly, subtract 129 * s * Sx
+//   uint4    w = s * (q - z)                     -> decode 128 + q exactly, subtract s * (128 + z) * Sx
+// where Sx is the sum of the group's X entries per token (an MMA against a ones operand). Each
+// product is exact in fp32, so the only roundings are the fp32 accumulations and the final bf16
+// store; no X conversion pass is needed.
+//
+// Work decomposition. A CTA (one per SM) owns 8 * NOCT weight rows (<= 128) and one K slice; the
+// K slices of a row block run on the CTAs of a thread-block cluster and are summed in rank
+// order through distributed shared memory. Tiles are visited persistently when there are more
+// row blocks than co-resident clusters. Inside a CTA:
+//   * 512-wide K steps stream through a shared-memory ring with TMA: the X slice [16 tokens]
+//     [512] (rows past M are zero-filled by the copy), the packed codes of the tile's rows and
+//     the scales (and zeros) of the step's groups. There is no producer warp: thread 0 issues
+//     the first ring's worth, and afterwards the last warp to finish with a slot refills it
+//     (a shared-memory arrival counter), so no warp ever blocks on a slot being released;
+//   * each of the eight warps takes 64 of the step's 512 K (one group or half of one): it turns
+//     its group's fp16 scales / zeros into fp32 pairs (s, s * c), loads its four X fragments
+//     once with ldmatrix, forms Sx with four MMAs against ones, and runs the decode + MMA
+//     chains of all the tile's octets, their codes loaded ahead of each sub-batch;
+//   * at the end of a tile the eight warps' partial sums are added in a fixed order through
+//     shared memory, then across the cluster, so results do not depend on timing.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "lowbit_internal.h"
+#include "sm100_ptx.cuh"
+
+namespace lowbit {
+namespace smallm {
+
+constexpr int kWarps = 8;                         // each takes 64 K of every step
+constexpr int kThreads = kWarps * 32;
+constexpr int kStepK = 512;                       // K per ring step
+constexpr int kTokens = 16;
+constexpr int kMaxRows = 128;
+constexpr int kMaxOct = kMaxRows / 8;
+constexpr int kMaxChains = 12;                    // octet chains interleaved per sub-batch
+constexpr int kMaxStages = 8;
+constexpr int kXBytes = kTokens * kStepK * 2;     // X slice of one step: 16 KB
+constexpr int kSmemLimit = 227 * 1024;
+constexpr int kBarBytes = 256;
+constexpr uint32_t kBf16One2 = 0x3F803F80u;       // bf16 pair (1, 1)
+
+template <int BITS, int GS>
+struct Fmt {
+    static constexpr int kGroups = kStepK / GS;              // scale rows per step
+    static constexpr int kWBoxes = BITS == 4 ? 2 : 1;        // TMA boxes of codes per step
+    static constexpr int kWRow = BITS == 1 ? 64 : 128;       // bytes per row per box
+    static constexpr int kWBoxWords = kWRow / 4;
+};
+
+struct Params {
+    int M, N, K;
+    int kslice, ksplit;   // K per cluster rank (multiple of 512) and ranks per cluster
+    int n_tiles;          // ceil(N / rows)
+    int stages;
+    uint32_t stage_bytes, w_off, s_off, z_off, tx_bytes;
+    uint32_t scr_off, red_off, part_off, bar_off;
+    __nv_bfloat16* Y;
+    unsigned* status;     // the device status word (bounded waits record timeouts here)
+};
+
+// Shared-memory layout for `rows` weight rows per tile. Every TMA destination starts on a
+// 128-byte boundary (1024 for the swizzled X and code boxes). Returns false if fewer than two
+// ring stages fit.
+template <int BITS, int GS>
+bool layout(int rows, int ksplit, Params* p, int* smem_bytes) {
+    using F = Fmt<BITS, GS>;
+    const int noct = rows / 8;
+    const uint32_t w_bytes = F::kWBoxes * rows * F::kWRow;   // a multiple of 512
+    const uint32_t s_raw = F::kGroups * rows * 2;
+    const uint32_t s_bytes = (s_raw + 127) / 128 * 128;
+    p->w_off = kXBytes;
+    p->s_off = p->w_off + w_bytes;
+    p->z_off = p->s_off + s_bytes;
+    const uint32_t end = p->z_off + (BITS == 4 ? s_bytes : 0);
+    p->stage_bytes = (end + 1023) / 1024 * 1024;
+    p->tx_bytes = kXBytes + w_bytes + s_raw * (BITS == 4 ? 2 : 1);
+    const uint32_t scr = kWarps * (rows / 2) * 16;   // per warp: (s, s * c) pairs of its group
+    const uint32_t red = 4 * noct * 512;
+    const uint32_t part = ksplit > 1 ? noct * 512 : 0;
+    const int fixed = static_cast<int>(scr + red + part) + kBarBytes + 1024;
+    int stages = (kSmemLimit - fixed) / static_cast<int>(p->stage_bytes);
+    if (stages > kMaxStages) stages = kMaxStages;
+    if (stages < 2) return false;
+    p->stages = stages;
+    p->scr_off = stages * p->stage_bytes;
+    p->red_off = p->scr_off + scr;
+    p->part_off = p->red_off + red;
+    p->bar_off = p->part_off + part;
+    *smem_bytes = static_cast<int>(p->bar_off) + kBarBytes + 1024;
+    return true;
+}
+
+// ---- device helpers -------------------------------------------------------------------------
+__device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t (&a)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
+                 : "r"(addr));
+}
+
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// The same with a zero accumulator input (first K step of a group sum).
+__device__ __forceinline__ void mma_bf16_z(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%10, %10, %10, %10};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.f));
+}
+
+__device__ __forceinline__ void cta_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
+// Shared-memory counter increment with acquire-release ordering at CTA scope; returns the old value.
+__device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t* p, uint32_t v) {
+    uint32_t old;
+    asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], %2;" : "=r"(old) : "r"(smem_u32(p)), "r"(v) : "memory");
+    return old;
+}
+
+// Arrive on the barrier at `cluster_addr` (a shared::cluster address), releasing this thread's
+// prior writes (and, through the preceding CTA barrier, its CTA's) at cluster scope.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait_acq_cluster(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait with cluster-scope acquire (for barriers other CTAs of the cluster arrive on).
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                                  unsigned* status_word) {
+    const long long t0 = clock64();
+    uint32_t it = 0;
+    while (!mbar_try_wait_acq_cluster(bar, parity)) {
+        if ((++it & 63u) == 0) {
+            if (*abort_flag) return false;
+            if (clock64() - t0 > kWaitLimitCycles) {
+                atomicOr(status_word, kDevErrTimeout);
+                *abort_flag = 1;
+                return false;
+            }
+        }
+    }
+    return true;
+}
+
+// Exact bf16 pairs of two neighbouring codes (k, k + 1) at pair index c of a packed word.
+__device__ __forceinline__ uint32_t dec_u4(uint32_t v, int c) {       // 128 + q
+    return and_or(v >> (4 * c), 0x000F000Fu, 0x43004300u);
+}
+__device__ __forceinline__ uint32_t dec_t2(uint32_t v, int c) {       // 128 + f, f = t + 1
+    return and_or(v >> (2 * c), 0x00030003u, 0x43004300u);
+}
+__device__ __forceinline__ uint32_t dec_b1(uint32_t v, int c) {       // +-1 by the code bit
+    return xor_andnot(0x3F803F80u, v << (15 - c), 0x80008000u);
+}
+
+template <int BITS, int GS, int NOCT>
+__global__ void __launch_bounds__(kThreads, 1)
+    lowbit_smallm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w,
+                         const __grid_constant__ CUtensorMap map_s, const __grid_constant__ CUtensorMap map_z,
+                         const Params p) {
+    using F = Fmt<BITS, GS>;
+    constexpr int R = 8 * NOCT;                       // weight rows per tile
+    constexpr int HALF = R / 2;                       // (s, s * c) pairs per group
+    constexpr int NB = (NOCT + kMaxChains - 1) / kMaxChains;
+    constexpr int B = (NOCT + NB - 1) / NB;           // octets per sub-batch
+    constexpr int WPS = BITS == 4 ? 8 : BITS == 2 ? 4 : 2;   // code words per lane per octet per step
+    if (threadIdx.x == 0) {
+        tma_prefetch_desc(&map_x);
+        tma_prefetch_desc(&map_w);
+        tma_prefetch_desc(&map_s);
+        if (BITS == 4) tma_prefetch_desc(&map_z);
+    }
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int S = p.stages;
+    uint8_t* ring = smem;
+    float4* red = reinterpret_cast<float4*>(smem + p.red_off);
+    float4* part = reinterpret_cast<float4*>(smem + p.part_off);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + p.bar_off);
+    uint64_t* pready = full + kMaxStages;      // every rank's part of the tile is written
+    uint64_t* pfree = pready + 1;              // every rank has read this CTA's part
+    uint32_t* cnt = reinterpret_cast<uint32_t*>(pfree + 1);   // per slot: warps done, all rounds
+    uint32_t* iss = cnt + kMaxStages;                         // per slot: fills issued
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(iss + kMaxStages);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int ks = p.ksplit;
+    const int rank = static_cast<int>(blockIdx.y);
+    const int k_begin = rank * p.kslice;
+    const int k_len = min(p.kslice, p.K - k_begin);   // > 0 by construction
+    const int nst = (k_len + kStepK - 1) / kStepK;
+    const int my_tiles = (p.n_tiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
+                         static_cast<int>(gridDim.x);
+    const int total = my_tiles * nst;                 // ring steps this CTA consumes
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kMaxStages; ++i) {
+            mbar_init(&full[i], 1);
+            cnt[i] = 0;
+            iss[i] = 0;
+        }
+        mbar_init(pready, ks);
+        mbar_init(pfree, ks);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (ks > 1) cluster_sync_all();   // other ranks arrive on this CTA's barriers
+    grid_launch_dependents();
+
+    // Ring step `gs` of this CTA: tile blockIdx.x + (gs / nst) * gridDim.x, K step gs % nst.
+    auto issue = [&](int gs, bool codes, bool x) {
+        const int s = gs % S;
+        uint8_t* st = ring + s * p.stage_bytes;
+        const int n0 = (static_cast<int>(blockIdx.x) + (gs / nst) * static_cast<int>(gridDim.x)) * R;
+        const int kk = k_begin + (gs % nst) * kStepK;
+        if (codes) {
+            mbar_arrive_expect_tx(&full[s], p.tx_bytes);
+#pragma unroll
+            for (int b = 0; b < F::kWBoxes; ++b)
+                tma_load_2d(&map_w, &full[s], st + p.w_off + b * R * F::kWRow, kk * BITS / 32 + b * F::kWBoxWords, n0);
+            tma_load_2d(&map_s, &full[s], st + p.s_off, n0, kk / GS);
+            if (BITS == 4) tma_load_2d(&map_z, &full[s], st + p.z_off, n0, kk / GS);
+        }
+        if (x) tma_load_3d(&map_x, &full[s], st, 0, 0, kk / 64);
+    };
+    // The codes, scales and zeros are not written by earlier kernels of the stream that this one
+    // may overlap: thread 0 fetches the first ring's share at once, while lane 0 of warp 1 waits
+    // for those kernels and then adds X, so step 0's X is queued right behind its codes.
+    const int pre = min(S, total);
+    if (threadIdx.x == 0) {
+        for (int gs = 0; gs < pre; ++gs) {
+            issue(gs, true, false);
+            iss[gs] = 1;
+        }
+    } else if (threadIdx.x == 32) {
+        grid_dependency_wait();
+        for (int gs = 0; gs < pre; ++gs) issue(gs, false, true);
+    }
+
+    const int w = warp;
+    const int g = lane >> 2;                 // B column (weight row in the octet) / C row
+    const int q = lane & 3;
+    const int gi = (w * 64) / GS;            // this warp's group within a step
+    const int tok = lane & 15;               // ldmatrix row (token) supplied by this lane
+    const uint32_t xoff = static_cast<uint32_t>(w * 2048 + tok * 128);
+    const int xhalf = lane >> 4;
+    // This lane's code bytes in row g of octet 0 of a step (swizzled as the TMA wrote them; the
+    // swizzle depends on the row only through g, so octet o is at a fixed offset from it).
+    uint32_t wb0, wb1;                       // two 16-byte pieces (uint4) or one piece (others)
+    constexpr uint32_t kOctStride = BITS == 1 ? 512u : 1024u;
+    if (BITS == 4) {
+        const int c0 = 2 * (w & 3);
+        wb0 = static_cast<uint32_t>((w >> 2) * R * 128 + g * 128 + ((c0 ^ g) << 4));
+        wb1 = static_cast<uint32_t>((w >> 2) * R * 128 + g * 128 + (((c0 + 1) ^ g) << 4));
+    } else if (BITS == 2) {
+        wb0 = wb1 = static_cast<uint32_t>(g * 128 + ((w ^ g) << 4));
+    } else {
+        wb0 = wb1 = static_cast<uint32_t>(g * 64 + (((w >> 1) ^ ((g >> 1) & 3)) << 4) + (w & 1) * 8);
+    }
+    float4* scr = reinterpret_cast<float4*>(smem + p.scr_off) + w * HALF;
+
+    float acc[NOCT][4];
+#pragma unroll
+    for (int o = 0; o < NOCT; ++o) acc[o][0] = acc[o][1] = acc[o][2] = acc[o][3] = 0.f;
+    int it = 0, ti = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < p.n_tiles; t += gridDim.x, ++ti) {
+        for (int c = 0; c < nst; ++c, ++it) {
+            const int s = it % S;
+            ok = ok && __all_sync(0xffffffffu, mbar_wait(&full[s], (it / S) & 1u, abort_flag, p.status));
+            if (ok) {
+                const uint8_t* st = ring + s * p.stage_bytes;
+                const uint32_t st_u = smem_u32(st);
+                // this warp's group: fp32 (s, s * c) for every pair of rows of the tile
+                {
+                    const __half2* sp = reinterpret_cast<const __half2*>(st + p.s_off) + gi * HALF;
+                    const __half2* zp = reinterpret_cast<const __half2*>(st + p.z_off) + gi * HALF;
+#pragma unroll
+                    for (int i0 = 0; i0 < HALF; i0 += 32) {
+                        const int i = i0 + lane;
+                        if (i < HALF) {
+                            const float2 sf = __half22float2(sp[i]);
+                            float c0 = 0.f, c1 = 0.f;
+                            if (BITS == 4) {
+                                const float2 zf = __half22float2(zp[i]);
+                                c0 = sf.x * (128.f + zf.x);
+                                c1 = sf.y * (128.f + zf.y);
+                            } else if (BITS == 2) {
+                                c0 = 129.f * sf.x;
+                                c1 = 129.f * sf.y;
+                            }
+                            scr[i] = make_float4(sf.x, sf.y, c0, c1);
+                        }
+                    }
+                    __syncwarp();
+                }
+                // X fragments of this warp's four 16-wide K steps (128-byte swizzled rows)
+                uint32_t a[4][4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int chunk = (j << 1) | xhalf;
+                    ldmatrix_x4(st_u + xoff + static_cast<uint32_t>((chunk ^ (tok & 7)) << 4), a[j]);
+                }
+                float tsx[4] = {0.f, 0.f, 0.f, 0.f};   // group sums of X: tokens g (0), g + 8 (2)
+                if (BITS != 1) {
+                    mma_bf16_z(tsx, a[0], kBf16One2, kBf16One2);
+#pragma unroll
+                    for (int j = 1; j < 4; ++j) mma_bf16(tsx, a[j], kBf16One2, kBf16One2);
+                }
+                const uint8_t* wst = st + p.w_off;
+#pragma unroll
+                for (int ob = 0; ob < NOCT; ob += B) {
+                    // codes of the sub-batch's octets for this warp's 64 K
+                    uint32_t wd[B][WPS];
+#pragma unroll
+                    for (int u = 0; u < B; ++u) {
+                        if (ob + u < NOCT) {
+                            const uint8_t* rp = wst + (ob + u) * kOctStride;
+                            if (BITS == 4) {
+                                const uint4 v0 = *reinterpret_cast<const uint4*>(rp + wb0);
+                                const uint4 v1 = *reinterpret_cast<const uint4*>(rp + wb1);
+                                wd[u][0] = v0.x; wd[u][1] = v0.y; wd[u][2] = v0.z; wd[u][3] = v0.w;
+                                wd[u][4] = v1.x; wd[u][5] = v1.y; wd[u][6] = v1.z; wd[u][7] = v1.w;
+                            } else if (BITS == 2) {
+                                const uint4 v = *reinterpret_cast<const uint4*>(rp + wb0);
+                                wd[u][0] = v.x; wd[u][1] = v.y; wd[u][2] = v.z; wd[u][3] = v.w;
+                            } else {
+                                const uint2 v = *reinterpret_cast<const uint2*>(rp + wb0);
+                                wd[u][0] = v.x; wd[u][1] = v.y;
+                            }
+                        }
+                    }
+                    float T[B][4];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+#pragma unroll
+                        for (int u = 0; u < B; ++u) {
+                            if (ob + u < NOCT) {
+                                uint32_t b0, b1;
+                                if (BITS == 4) {
+                                    b0 = dec_u4(wd[u][2 * j], q);
+                                    b1 = dec_u4(wd[u][2 * j + 1], q);
+                                } else if (BITS == 2) {
+                                    b0 = dec_t2(wd[u][j], q);
+                                    b1 = dec_t2(wd[u][j], q + 4);
+                                } else {
+                                    const int pc = (j & 1) * 8 + q;
+                                    b0 = dec_b1(wd[u][j >> 1], pc);
+                                    b1 = dec_b1(wd[u][j >> 1], pc + 4);
+                                }
+                                if (j == 0) mma_bf16_z(T[u], a[0], b0, b1);
+                                else mma_bf16(T[u], a[j], b0, b1);
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int u = 0; u < B; ++u) {
+                        if (ob + u < NOCT) {
+                            const float4 sc = scr[4 * (ob + u) + q];
+                            float* d = acc[ob + u];
+                            d[0] = fmaf(sc.x, T[u][0], d[0]);
+                            d[1] = fmaf(sc.y, T[u][1], d[1]);
+                            d[2] = fmaf(sc.x, T[u][2], d[2]);
+                            d[3] = fmaf(sc.y, T[u][3], d[3]);
+                            if (BITS != 1) {
+                                d[0] = fmaf(-sc.z, tsx[0], d[0]);
+                                d[1] = fmaf(-sc.w, tsx[0], d[1]);
+                                d[2] = fmaf(-sc.z, tsx[2], d[2]);
+                                d[3] = fmaf(-sc.w, tsx[2], d[3]);
+                            }
+                        }
+                    }
+                }
+            }
+            __syncwarp();
+            // Release the slot; the last warp out refills it with ring step it + S.
+            if (lane == 0) {
+                const uint32_t prev = atom_add_acq_rel(&cnt[s], 1);
+                if ((prev & (kWarps - 1)) == kWarps - 1 && it + S < total && !*abort_flag) {
+                    issue(it + S, true, true);
+                    iss[s] += 1;
+                }
+            }
+        }
+
+        // ---- tile end: sum the eight warps' partials in a fixed order: (w + (w + 4)) for
+        // w < 4, then ((0 + 1) + 2) + 3.
+        grid_dependency_wait();   // Y may still be read by the kernel this one overlaps
+        cta_bar();                // the previous tile's readers of `red` are done
+        if (w >= 4) {
+#pragma unroll
+            for (int o = 0; o < NOCT; ++o)
+                red[((w - 4) * NOCT + o) * 32 + lane] = make_float4(acc[o][0], acc[o][1], acc[o][2], acc[o][3]);
+        }
+        cta_bar();
+        if (w < 4) {
+#pragma unroll
+            for (int o = 0; o < NOCT; ++o) {
+                const float4 v = red[(w * NOCT + o) * 32 + lane];
+                acc[o][0] += v.x;
+                acc[o][1] += v.y;
+                acc[o][2] += v.z;
+                acc[o][3] += v.w;
+            }
+        }
+        cta_bar();
+        if (w < 4) {
+#pragma unroll
+            for (int o = 0; o < NOCT; ++o)
+                red[(w * NOCT + o) * 32 + lane] = make_float4(acc[o][0], acc[o][1], acc[o][2], acc[o][3]);
+        }
+        cta_bar();
+#pragma unroll
+        for (int o = 0; o < NOCT; ++o) acc[o][0] = acc[o][1] = acc[o][2] = acc[o][3] = 0.f;
+
+        const int n0 = t * R;
+        auto store = [&](int o, float4 v) {
+            const int n = n0 + 8 * o + 2 * q;
+            if (n < p.N) {
+                if (g < p.M)
+                    *reinterpret_cast<__nv_bfloat162*>(p.Y + static_cast<size_t>(g) * p.N + n) =
+                        __floats2bfloat162_rn(v.x, v.y);
+                if (g + 8 < p.M)
+                    *reinterpret_cast<__nv_bfloat162*>(p.Y + static_cast<size_t>(g + 8) * p.N + n) =
+                        __floats2bfloat162_rn(v.z, v.w);
+            }
+        };
+        auto tile_sum = [&](int o) {
+            float4 v = red[o * 32 + lane];
+#pragma unroll
+            for (int r = 1; r < 4; ++r) {
+                const float4 u = red[(r * NOCT + o) * 32 + lane];
+                v.x += u.x;
+                v.y += u.y;
+                v.z += u.z;
+                v.w += u.w;
+            }
+            return v;
+        };
+        if (ks == 1) {
+            for (int o = w; o < NOCT; o += kWarps) store(o, tile_sum(o));
+        } else {
+            // publish this rank's tile sums, then rank r finishes the octets o with o % ks == r,
+            // adding the ranks' sums in rank order (all remote loads issued before the sum)
+            if (ti > 0)
+                ok = __all_sync(0xffffffffu, mbar_wait_cluster(pfree, (ti - 1) & 1u, abort_flag, p.status)) && ok;
+            for (int o = w; o < NOCT; o += kWarps) part[o * 32 + lane] = tile_sum(o);
+            cta_bar();
+            if (threadIdx.x == 0)
+                for (int r = 0; r < ks; ++r) mbar_arrive_cluster(map_shared_rank(smem_u32(pready), r));
+            ok = __all_sync(0xffffffffu, mbar_wait_cluster(pready, ti & 1u, abort_flag, p.status)) && ok;
+            for (int o = w; o < NOCT; o += kWarps) {
+                if (o % ks != rank) continue;
+                const uint32_t addr = smem_u32(part + o * 32 + lane);
+                float4 v[8];
+#pragma unroll
+                for (int r = 0; r < 8; ++r)
+                    if (r < ks) v[r] = ld_shared_cluster_v4(map_shared_rank(addr, r));
+                float4 sum = v[0];
+#pragma unroll
+                for (int r = 1; r < 8; ++r)
+                    if (r < ks) {
+                        sum.x += v[r].x;
+                        sum.y += v[r].y;
+                        sum.z += v[r].z;
+                        sum.w += v[r].w;
+                    }
+                store(o, sum);
+            }
+            cta_bar();
+            if (threadIdx.x == 0)
+                for (int r = 0; r < ks; ++r) mbar_arrive_cluster(map_shared_rank(smem_u32(pfree), r));
+        }
+    }
+    // Stay resident until every rank has read this CTA's last partial sums, and leave no copy in
+    // flight into shared memory (only possible after an aborted wait).
+    if (ks > 1 && ti > 0) mbar_wait_cluster(pfree, (ti - 1) & 1u, abort_flag, p.status);
+    cta_bar();
+    if (threadIdx.x == 0 && *abort_flag) {
+        int zero = 0;
+        for (int i = 0; i < S; ++i)
+            if (iss[i]) mbar_wait(&full[i], (iss[i] - 1) & 1u, &zero, p.status, kWaitLimitCycles / 8);
+    }
+}
+
+// Kernel entry for (BITS, GS) and `noct` octets per tile (1..16), or nullptr. One definition
+// per code width lives in its own translation unit so the instantiations build in parallel.
+const void* kernel_b1(int group_size, int noct);
+const void* kernel_b2(int group_size, int noct);
+const void* kernel_b4(int group_size, int noct);
+
+}  // namespace smallm
+}  // namespace lowbit
+
+// Defines kernel_b<BITS>: a table of the sixteen octet counts for both group sizes.
+#define LOWBIT_SMALLM_TABLE(BITS)                                                                     \
+    namespace lowbit {                                                                                \
+    namespace smallm {                                                                                \
+    template <int GS, int... Ns>                                                                      \
+    static const void* pick_##BITS(int noct, std::integer_sequence<int, Ns...>) {                     \
+        static const void* const table[] = {                                                          \
+            reinterpret_cast<const void*>(&lowbit_smallm_kernel<BITS, GS, Ns + 1>)...};               \
+        return (noct >= 1 && noct <= static_cast<int>(sizeof...(Ns))) ? table[noct - 1] : nullptr;    \
+    }                                                                                                 \
+    const void* kernel_b##BITS(int group_size, int noct) {                                            \
+        if (group_size == 64) return pick_##BITS<64>(noct, std::make_integer_sequence<int, kMaxOct>{}); \
+        if (group_size == 128) return pick_##BITS<128>(noct, std::make_integer_sequence<int, kMaxOct>{}); \
+        return nullptr;                                                                               \
+    }                                                                                                 \
+    }                                                                                                 \
+    }

@@ -110,11 +110,13 @@ lowbit_status lowbit_gemm(int64_t M, int64_t N, int64_t K, int bits, int group_s
 /* lowbit_gemm with the kernel configuration fixed instead of chosen from the shape, for
  * tuning and tests (each 0 = automatic):
  *   tile_tokens  tokens per CTA tile of the tensor-memory kernel: 16, 32, 64, 128 or 256; or 1
- *                for the small-M kernel on warp-level MMAs (M <= 16, tile_rows 0, K at most
- *                10240; chosen automatically for M <= 16)
+ *                for the small-M kernel on warp-level MMAs (M <= 16 only; chosen automatically
+ *                for M <= 16; it reads X directly and leaves the workspace untouched)
  *   tile_rows    weight rows per CTA tile: a multiple of 8 up to 128 (128 unless the shape is
  *                small; fewer rows give more CTAs, each streaming the whole K)
- *   ksplit       number of K slices summed across a thread-block cluster, 1..8 (1 = no split)
+ *   ksplit       number of K slices summed across a thread-block cluster, 1..8 (1 = no split;
+ *                the small-M kernel cuts K into slices of whole 512-wide steps, so a request
+ *                may be served with fewer slices)
  * Other arguments and all checks are those of lowbit_gemm; values outside these sets return
  * LOWBIT_ERR_UNSUPPORTED. */
 lowbit_status lowbit_gemm_ex(int64_t M, int64_t N, int64_t K, int bits, int group_size, const void* X,

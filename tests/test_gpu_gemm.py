@@ -93,19 +93,38 @@ def test_gemm_flat_row_tiles(bits, gs, tile_tokens, tile_rows):
 
 @pytest.mark.parametrize("bits,gs", FORMATS)
 @pytest.mark.parametrize("M", [1, 5, 16])
-@pytest.mark.parametrize("K,N,ksplit", [(256, 520, 1), (192 * 4, 264, 3), (2560, 1032, 0), (9728, 256, 0)])
-def test_gemm_small_m_warp_mma(bits, gs, M, K, N, ksplit):
-    """The small-M kernel (warp-level MMAs, K split over a cluster), ragged N, partial k-blocks."""
+@pytest.mark.parametrize("K,N,rows,ksplit", [
+    (256, 520, 0, 1),       # one step, half of it past K
+    (768, 264, 0, 3),       # a request for 3 slices served with 2 (slices are whole 512-wide steps)
+    (2560, 1032, 0, 0),     # automatic choice
+    (9728, 256, 0, 0),      # long K, few rows: split over a cluster
+    (640, 136, 56, 0),      # 7 octets: a partial batch of four
+    (1152, 1000, 120, 2),   # the second slice holds one 128-wide group of K
+    (1024, 2376, 8, 1),     # more row blocks than SMs: persistent tiles, no cluster
+    (2048, 1352, 8, 2),     # persistent tiles with the cross-rank reduction on every tile
+])
+def test_gemm_small_m_warp_mma(bits, gs, M, K, N, rows, ksplit):
+    """The small-M kernel (warp-level MMAs on X as stored), ragged N and K, forced tilings."""
     if bits == 1 and K % 128:
         pytest.skip("binary needs K % 128 == 0")
     spec = spec_for(bits, gs, M, K, N, seed=M * 7 + K)
     prob = synth.make_problem(spec)
     ref = oracle.gemm(prob.x_bf16, _gpu.oracle_packed(prob), prob.scales, prob.zeros, N, bits, gs)
     x, packed, s, z = _gpu.dev_problem(prob)
-    y = lb.gemm(x, packed, s, z, bits, gs, tile_tokens=1, ksplit=ksplit)
+    y = lb.gemm(x, packed, s, z, bits, gs, tile_tokens=1, tile_rows=rows, ksplit=ksplit)
     torch.cuda.synchronize()
     assert lb.device_status() == 0
-    _gpu.check_close(_gpu.y_to_f64(y), ref, what=f"warp-mma M={M} K={K} N={N} split={ksplit}")
+    _gpu.check_close(_gpu.y_to_f64(y), ref, what=f"warp-mma M={M} K={K} N={N} rows={rows} split={ksplit}")
+
+
+def test_gemm_small_m_deterministic():
+    """Repeated small-M runs with a cluster split give bit-identical outputs (fixed summation order)."""
+    spec = spec_for(4, 64, 16, 9728, 2560, seed=5)
+    prob = synth.make_problem(spec)
+    x, packed, s, z = _gpu.dev_problem(prob)
+    ys = [lb.gemm(x, packed, s, z, 4, 64, tile_tokens=1, ksplit=4).clone() for _ in range(3)]
+    torch.cuda.synchronize()
+    assert all(torch.equal(ys[0].view(torch.int16), y.view(torch.int16)) for y in ys[1:])
 
 
 def test_gemm_small_m_k_partial_block():
