@@ -102,7 +102,8 @@ bool layout(int rows, int ksplit, Params* p, int* smem_bytes) {
     p->tx_bytes = kXBytes + w_bytes + s_raw * (BITS == 4 ? 2 : 1);
     const uint32_t scr = kWarps * (rows / 2) * 16;   // per warp: (s, s * c) pairs of its group
     const uint32_t red = 4 * noct * 512;
-    const uint32_t part = ksplit > 1 ? noct * 512 : 0;
+    // receive buffer of the octets this rank finishes: [ksplit][ceil(noct / ksplit)][32 lanes]
+    const uint32_t part = ksplit > 1 ? ksplit * ((noct + ksplit - 1) / ksplit) * 512 : 0;
     const int fixed = static_cast<int>(scr + red + part) + kBarBytes + 1024;
     int stages = (kSmemLimit - fixed) / static_cast<int>(p->stage_bytes);
     if (stages > kMaxStages) stages = kMaxStages;
@@ -149,10 +150,20 @@ __device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t* p, uint32_t v) {
     return old;
 }
 
-// Arrive on the barrier at `cluster_addr` (a shared::cluster address), releasing this thread's
-// prior writes (and, through the preceding CTA barrier, its CTA's) at cluster scope.
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+// Makes this thread's prior writes (and, through the preceding CTA barrier, its CTA's) visible
+// at cluster scope before the relaxed arrivals that follow it.
+__device__ __forceinline__ void fence_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
+
+// Arrive on the barrier at `cluster_addr` (a shared::cluster address) without ordering; pair
+// with fence_cluster().
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+__device__ __forceinline__ void st_shared_cluster_v4(uint32_t addr, float4 v) {
+    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.x), "f"(v.y), "f"(v.z),
+                 "f"(v.w)
+                 : "memory");
 }
 
 __device__ __forceinline__ bool mbar_try_wait_acq_cluster(uint64_t* bar, uint32_t parity) {
@@ -337,7 +348,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             scr[i] = make_float4(sf.x, sf.y, c0, c1);
                         }
                     }
-                    __syncwarp();
+                    // (read back by the other lanes only after the first sub-batch's MMAs)
                 }
                 // X fragments of this warp's four 16-wide K steps (128-byte swizzled rows)
                 uint32_t a[4][4];
@@ -398,6 +409,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             }
                         }
                     }
+                    if (ob == 0) __syncwarp();   // the scale pairs above are written
 #pragma unroll
                     for (int u = 0; u < B; ++u) {
                         if (ob + u < NOCT) {
@@ -485,36 +497,43 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ks == 1) {
             for (int o = w; o < NOCT; o += kWarps) store(o, tile_sum(o));
         } else {
-            // publish this rank's tile sums, then rank r finishes the octets o with o % ks == r,
-            // adding the ranks' sums in rank order (all remote loads issued before the sum)
+            // Octet o is finished by rank o % ks: every rank stores its tile sum of o straight into
+            // that rank's receive buffer (slot [own rank][o / ks]), then the finishing rank adds
+            // the slots in rank order. pready: all ranks' sums have landed here; pfree: every
+            // finishing rank has consumed what this rank sent, so its buffers may be reused.
+            const int per = (NOCT + ks - 1) / ks;
             if (ti > 0)
                 ok = __all_sync(0xffffffffu, mbar_wait_cluster(pfree, (ti - 1) & 1u, abort_flag, p.status)) && ok;
-            for (int o = w; o < NOCT; o += kWarps) part[o * 32 + lane] = tile_sum(o);
+            for (int o = w; o < NOCT; o += kWarps) {
+                const uint32_t slot = smem_u32(part + ((rank * per + o / ks) * 32 + lane));
+                st_shared_cluster_v4(map_shared_rank(slot, o % ks), tile_sum(o));
+            }
             cta_bar();
-            if (threadIdx.x == 0)
-                for (int r = 0; r < ks; ++r) mbar_arrive_cluster(map_shared_rank(smem_u32(pready), r));
+            if (threadIdx.x == 0) {
+                fence_cluster();
+                for (int r = 0; r < ks; ++r) mbar_arrive_cluster_relaxed(map_shared_rank(smem_u32(pready), r));
+            }
             ok = __all_sync(0xffffffffu, mbar_wait_cluster(pready, ti & 1u, abort_flag, p.status)) && ok;
             for (int o = w; o < NOCT; o += kWarps) {
                 if (o % ks != rank) continue;
-                const uint32_t addr = smem_u32(part + o * 32 + lane);
-                float4 v[8];
-#pragma unroll
-                for (int r = 0; r < 8; ++r)
-                    if (r < ks) v[r] = ld_shared_cluster_v4(map_shared_rank(addr, r));
-                float4 sum = v[0];
+                const int li = o / ks;
+                float4 sum = part[li * 32 + lane];
 #pragma unroll
                 for (int r = 1; r < 8; ++r)
                     if (r < ks) {
-                        sum.x += v[r].x;
-                        sum.y += v[r].y;
-                        sum.z += v[r].z;
-                        sum.w += v[r].w;
+                        const float4 v = part[(r * per + li) * 32 + lane];
+                        sum.x += v.x;
+                        sum.y += v.y;
+                        sum.z += v.z;
+                        sum.w += v.w;
                     }
                 store(o, sum);
             }
             cta_bar();
-            if (threadIdx.x == 0)
-                for (int r = 0; r < ks; ++r) mbar_arrive_cluster(map_shared_rank(smem_u32(pfree), r));
+            if (threadIdx.x == 0) {
+                fence_cluster();
+                for (int r = 0; r < ks; ++r) mbar_arrive_cluster_relaxed(map_shared_rank(smem_u32(pfree), r));
+            }
         }
     }
     // Stay resident until every rank has read this CTA's last partial sums, and leave no copy in
