@@ -106,9 +106,13 @@ class ClockSampler:
 # --------------------------------------------------------------------------------------------
 # workload setup
 # --------------------------------------------------------------------------------------------
-def setup(specs, device, lb, torch, pinned=True):
+def setup(specs, device, lb, torch, pinned=True, copies=1):
     """Device inputs / outputs for every linear (weights packed on the GPU by the library),
-    plus pinned host copies of the activations and host buffers for the outputs."""
+    plus pinned host copies of the activations and host buffers for the outputs.
+
+    copies > 1 gives each linear that many distinct device copies of its packed weights, scales
+    and zeros (same values), used in rotation so that a workload smaller than L2 still streams
+    its weights from HBM every step. Returns (items, descriptor lists, one per copy)."""
     items = []
     for spec in specs:
         prob = synth.make_problem(spec)
@@ -123,10 +127,17 @@ def setup(specs, device, lb, torch, pinned=True):
         z = torch.from_numpy(prob.zeros).to(device) if prob.zeros is not None else None
         y = torch.empty((spec.M, spec.N), dtype=torch.bfloat16, device=device)
         y_host = torch.empty((spec.M, spec.N), dtype=torch.bfloat16, pin_memory=pinned)
-        items.append(dict(spec=spec, x=x, packed=packed, s=s, z=z, y=y, x_host=x_host, y_host=y_host))
-    descs = [lb.make_desc(it["x"], it["packed"], it["s"], it["z"], it["y"], it["spec"].bits,
-                          it["spec"].group_size) for it in items]
-    return items, descs
+        reps = [(packed, s, z)] + [(packed.clone(), s.clone(), z.clone() if z is not None else None)
+                                   for _ in range(copies - 1)]
+        items.append(dict(spec=spec, x=x, packed=packed, s=s, z=z, y=y, x_host=x_host, y_host=y_host, reps=reps))
+    desc_sets = [[lb.make_desc(it["x"], it["reps"][c][0], it["reps"][c][1], it["reps"][c][2], it["y"],
+                               it["spec"].bits, it["spec"].group_size) for it in items] for c in range(copies)]
+    return items, desc_sets
+
+
+def weight_bytes(specs):
+    """Packed codes + scales (+ zeros) of the workload: what streams from HBM every step."""
+    return sum(s.algorithmic_bytes() - s.M * s.K * 2 - s.M * s.N * 2 for s in specs)
 
 
 def step_flops(specs):
@@ -229,10 +240,22 @@ def run_lowbit(args, specs, workload):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(specs, args.ref_rows)   # before any timed GPU work; uses host cores only
 
-    items, descs = setup(specs, device, lb, torch, pinned=not args.no_e2e)
     flops = step_flops(specs)
     nbytes = step_bytes(specs)
+    l2_bytes = torch.cuda.get_device_properties(device).L2_cache_size
+    # A workload that fits in L2 rotates distinct copies of its weights (at least 20, and enough
+    # to exceed twice L2) so that every step reads them from HBM, with no flush between steps.
+    copies = 1
+    if nbytes < 2 * l2_bytes:
+        copies = min(256, max(20, -(-int(2.2 * l2_bytes) // max(1, weight_bytes(specs)))))
+    items, desc_sets = setup(specs, device, lb, torch, pinned=not args.no_e2e, copies=copies)
+    descs = desc_sets[0]
     stream = torch.cuda.current_stream(device)
+    peaks, peak_src = load_peaks()
+    # bound of the workload: below the ridge point (peak flop/s per peak byte/s) it is HBM-bound
+    ridge = peaks.get("bf16_tflops", 1590.0) * 1e12 / (peaks.get("hbm_gbs", 6650.0) * 1e9)
+    hbm_bound = flops / nbytes < ridge
+    launches_per_step = sum(1 if s.M <= 16 else 2 for s in specs)   # X conversion + GEMM above 16 tokens
 
     def barrier():
         if world > 1:
@@ -245,15 +268,29 @@ def run_lowbit(args, specs, workload):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         return float(t.item())
 
-    # single-linear workloads fit in L2: flush it (write a buffer larger than L2) between steps
-    l2_bytes = torch.cuda.get_device_properties(device).L2_cache_size
-    need_flush = nbytes < 2 * l2_bytes
-    flush = torch.empty(int(max(2 * l2_bytes, 256 << 20)), dtype=torch.uint8, device=device) if need_flush else None
+    # Each step is one lowbit_gemm_batch over the workload's linears, captured once per weight
+    # copy as a CUDA graph and replayed, so the timed region measures the GPU rather than the
+    # host's per-call submission cost (the end-to-end number below calls the API directly).
+    lb.gemm_batch(desc_sets[0], device)   # allocates the shared workspace before capture
+    torch.cuda.synchronize(device)
+    graphs = []
+    cap_stream = torch.cuda.Stream(device)
+    cap_stream.wait_stream(stream)
+    with torch.cuda.stream(cap_stream):
+        for c in range(copies):
+            gph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gph, stream=cap_stream):
+                lb.gemm_batch(desc_sets[c], device)
+            graphs.append(gph)
+    stream.wait_stream(cap_stream)
+    torch.cuda.synchronize(device)
+    step_idx = [0]
 
     def one_step():
-        lb.gemm_batch(descs, device)
+        graphs[step_idx[0] % copies].replay()
+        step_idx[0] += 1
 
-    for _ in range(args.warmup):
+    for _ in range(max(args.warmup, copies if copies > 1 else 0)):
         one_step()
     torch.cuda.synchronize(device)
     if lb.device_status() != 0:
@@ -263,23 +300,13 @@ def run_lowbit(args, specs, workload):
     clocks.start()
     barrier()
     torch.cuda.synchronize(device)
-    if need_flush:
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-        for a, b in evs:
-            flush.zero_()
-            a.record(stream)
-            one_step()
-            b.record(stream)
-        torch.cuda.synchronize(device)
-        ms_total = sum(a.elapsed_time(b) for a, b in evs)
-    else:
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(args.steps):
-            one_step()
-        b.record(stream)
-        torch.cuda.synchronize(device)
-        ms_total = a.elapsed_time(b)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.steps):
+        one_step()
+    b.record(stream)
+    torch.cuda.synchronize(device)
+    ms_total = a.elapsed_time(b)
     barrier()
     clk = clocks.stop()
     ms_total = max_over_ranks(ms_total)
@@ -288,21 +315,39 @@ def run_lowbit(args, specs, workload):
     if lb.device_status() != 0:
         raise RuntimeError("kernel timeout reported during the timed steps")
 
-    # per-launch durations of the (single) GEMM kernel, for the roofline: each linear timed on
-    # the launching stream with its own events, over two passes
+    # Per-launch durations for the roofline. Tensor-bound workloads: each linear timed on the
+    # launching stream with its own events, over two passes (inputs larger than L2). HBM-bound
+    # workloads: the launches run back to back over rotating weight copies, as in the timed
+    # steps, and a launch's duration is the pass time over the number of linears.
+    # Each distinct linear is captured `reps` times back to back in one graph (rotating weight
+    # copies where there are several) and the graph is replayed twice; a launch's duration is
+    # the replay time over `reps`. Each launch is one lowbit_gemm call: for more than 16 tokens
+    # that is the X conversion pass plus the GEMM kernel, for at most 16 the GEMM kernel alone.
     per = []
-    for _ in range(2):
-        evs = []
-        for it in items:
-            if need_flush:
-                flush.zero_()
+    seen = {}
+    for it in items:
+        seen.setdefault((it["spec"].M, it["spec"].K, it["spec"].N), it)
+    for it in seen.values():
+        reps = max(10, copies)
+        gph = torch.cuda.CUDAGraph()
+        cap_stream.wait_stream(stream)
+        with torch.cuda.stream(cap_stream):
+            with torch.cuda.graph(gph, stream=cap_stream):
+                for i in range(reps):
+                    w_p, w_s, w_z = it["reps"][i % copies]
+                    lb.gemm(it["x"], w_p, w_s, w_z, it["spec"].bits, it["spec"].group_size, out=it["y"])
+        stream.wait_stream(cap_stream)
+        gph.replay()
+        torch.cuda.synchronize(device)
+        for _ in range(2):
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-            lb.gemm(it["x"], it["packed"], it["s"], it["z"], it["spec"].bits, it["spec"].group_size, out=it["y"])
+            gph.replay()
             e1.record(stream)
-            evs.append((it["spec"], e0, e1))
-        torch.cuda.synchronize(device)
-        per.extend((sp, e0.elapsed_time(e1)) for sp, e0, e1 in evs)
+            torch.cuda.synchronize(device)
+            ms = e0.elapsed_time(e1) / reps
+            per.extend((sp, ms) for sp in [s for s in specs if (s.M, s.K, s.N) == (it["spec"].M, it["spec"].K, it["spec"].N)])
+        del gph
     launch_ms = sum(ms for _, ms in per) / len(per)
     launch_flops = sum(sp.flops for sp, _ in per) / len(per)
     launch_bytes = sum(sp.algorithmic_bytes() for sp, _ in per) / len(per)
@@ -315,7 +360,7 @@ def run_lowbit(args, specs, workload):
         for _ in range(1):
             for it in items:
                 it["x"].copy_(it["x_host"], non_blocking=True)
-            one_step()
+            lb.gemm_batch(descs, device)
             for it in items:
                 it["y_host"].copy_(it["y"], non_blocking=True)
         torch.cuda.synchronize(device)
@@ -326,7 +371,7 @@ def run_lowbit(args, specs, workload):
         for _ in range(e2e_steps):
             for it in items:
                 it["x"].copy_(it["x_host"], non_blocking=True)
-            one_step()
+            lb.gemm_batch(descs, device)
             for it in items:
                 it["y_host"].copy_(it["y"], non_blocking=True)
         b.record(stream)
@@ -335,17 +380,27 @@ def run_lowbit(args, specs, workload):
         e2e = {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_steps}
 
-    peaks, peak_src = load_peaks()
     long_step = ms_step >= 5.0
-    peak_tf = peaks.get("bf16_tflops_sustained" if long_step else "bf16_tflops")
-    achieved = launch_flops / (launch_ms * 1e-3) / 1e12
-    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
-                "frac": achieved / peak_tf, "traffic": None,
-                "peak_source": f"{peak_src} {'sustained' if long_step else 'burst'} bf16 dense",
-                "kernel": "lowbit_gemm_kernel", "launches_timed": len(per),
-                "algorithmic_gflop_per_launch": launch_flops / 1e9,
-                "algorithmic_mb_per_launch": launch_bytes / 1e6,
-                "frac_of_burst_peak": achieved / peaks.get("bf16_tflops", peak_tf)}
+    if hbm_bound:
+        peak_bw = peaks.get("hbm_gbs")
+        achieved = launch_bytes / (launch_ms * 1e-3) / 1e9
+        roofline = {"bound": "hbm", "achieved": achieved, "peak": peak_bw, "unit": "GB/s",
+                    "frac": achieved / peak_bw, "traffic": None,
+                    "peak_source": f"{peak_src} HBM copy bandwidth", "kernel": "lowbit_smallm_kernel",
+                    "launches_timed": len(per), "algorithmic_mb_per_launch": launch_bytes / 1e6,
+                    "algorithmic_gflop_per_launch": launch_flops / 1e9,
+                    "tflops_per_launch": launch_flops / (launch_ms * 1e-3) / 1e12,
+                    "weight_copies_rotated": copies}
+    else:
+        peak_tf = peaks.get("bf16_tflops_sustained" if long_step else "bf16_tflops")
+        achieved = launch_flops / (launch_ms * 1e-3) / 1e12
+        roofline = {"bound": "tensor", "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
+                    "frac": achieved / peak_tf, "traffic": None,
+                    "peak_source": f"{peak_src} {'sustained' if long_step else 'burst'} bf16 dense",
+                    "kernel": "lowbit_gemm_kernel", "launches_timed": len(per),
+                    "algorithmic_gflop_per_launch": launch_flops / 1e9,
+                    "algorithmic_mb_per_launch": launch_bytes / 1e6,
+                    "frac_of_burst_peak": achieved / peaks.get("bf16_tflops", peak_tf)}
 
     if rank == 0:
         spec0 = specs[0]
@@ -353,14 +408,17 @@ def run_lowbit(args, specs, workload):
                "group_size": spec0.group_size, "gflop_per_step": flops / 1e9,
                "algorithmic_mb_per_step": nbytes / 1e6,
                "shapes_MKN": sorted({(s.M, s.K, s.N) for s in specs}),
-               "l2": "flushed between steps (256+ MB write)" if need_flush else "inputs larger than L2 (no flush)",
+               "l2": (f"{copies} rotating copies of the weights ({copies * weight_bytes(specs) / 1e6:.0f} MB, "
+                      f"over 2x L2; no flush)") if copies > 1 else "inputs larger than L2 (no flush)",
                "parallelism": "replicas" if world > 1 else "single GPU"}
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
                 "hbm_gbs": world * nbytes / (ms_step * 1e-3) / 1e9,
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": len(specs) * args.steps, "clocks": clk}
+                "gpu_launches": launches_per_step * args.steps, "clocks": clk}
+        if len(specs) >= 40:   # a denoise step's chain: the pages count 4 steps per image
+            line["config"]["ms_per_4_steps"] = 4 * ms_step
         print(json.dumps(line), flush=True)
         if args.per_shape:
             agg = {}
@@ -372,7 +430,7 @@ def run_lowbit(args, specs, workload):
                 t = statistics.median(v)
                 print(f"# shape M={m} K={kk} N={n}: {t * 1e3:.1f} us, {2 * m * kk * n / t / 1e9:.1f} TFLOP/s",
                       file=sys.stderr)
-    del items, descs
+    del graphs, items, descs
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
