@@ -45,6 +45,8 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <mutex>
+
 #include <cstdint>
 #include <cstdio>
 
@@ -771,6 +773,40 @@ bool make_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, int elem_bytes, co
     return r == CUDA_SUCCESS;
 }
 
+int cluster_capacity(const void* kernel, int ks, int threads, int smem_bytes) {
+    struct Entry {
+        const void* fn;
+        int ks, cap;
+    };
+    static Entry cache[64];
+    static int used = 0;
+    static std::mutex mu;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        for (int i = 0; i < used; ++i)
+            if (cache[i].fn == kernel && cache[i].ks == ks) return cache[i].cap;
+    }
+    int n = 0;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = ks;
+    cfg.gridDim = dim3(1, 1, ks);
+    cfg.blockDim = dim3(threads, 1, 1);
+    cfg.dynamicSmemBytes = smem_bytes;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess || n <= 0) {
+        cudaGetLastError();
+        n = num_sms() / ks;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if (used < 64) cache[used++] = Entry{kernel, ks, n};
+    return n;
+}
+
 int num_sms() {
     static int sms = 0;
     if (!sms) {
@@ -827,6 +863,21 @@ lowbit_status launch(const GemmProblem& g, int rows, int ksplit_request, cudaStr
     p.Y = static_cast<__nv_bfloat16*>(g.Y);
     p.rowmul = rowmul;
     int ksplit = ksplit_request;
+    if (ksplit < 0) {
+        // Automatic: the largest split that leaves every rank at least 24 k-blocks (3072 of K)
+        // and keeps all clusters resident at once (the split grid is not persistent, so a
+        // second wave would double the time); cluster placement is limited by the GPC layout.
+        ksplit = 1;
+        const int slots = num_sms() * C::kCtasPerSm;
+        for (int ks = 8; ks >= 2; --ks) {
+            if (p.num_kb / ks < 24 || p.num_tiles * ks > slots) continue;
+            if (p.num_tiles <= cluster_capacity(reinterpret_cast<const void*>(kernel), ks, C::kThreads,
+                                                C::kSmemBytes)) {
+                ksplit = ks;
+                break;
+            }
+        }
+    }
     if (ksplit < 1) ksplit = 1;
     if (ksplit > 8) ksplit = 8;
     if (ksplit > p.num_kb) ksplit = p.num_kb;
@@ -916,16 +967,19 @@ lowbit_status gemm_launch(const GemmProblem& g, int force_bt, int force_rows, in
         ksplit = 1;
         if (bt <= 64 && m_tiles == 1 && flat_rows < kBlockN && x_per_w <= 1.25) {
             rows = static_cast<int>(flat_rows);
-        } else if (tiles128 * 2 <= slots && num_kb >= 4) {
-            const int64_t target = (bt <= 64 && m_tiles == 1) ? sms : slots;   // small M: one CTA per SM
-            int64_t s = target / tiles128;
-            if (s > 8) s = 8;
-            if (s > num_kb / 2) s = num_kb / 2;
-            ksplit = static_cast<int>(s < 1 ? 1 : s);
+        } else if (bt <= 64 && m_tiles == 1) {
+            if (tiles128 * 2 <= slots && num_kb >= 4) {
+                int64_t s = sms / tiles128;   // small M: one CTA per SM
+                if (s > 8) s = 8;
+                if (s > num_kb / 2) s = num_kb / 2;
+                ksplit = static_cast<int>(s < 1 ? 1 : s);
+            }
+        } else {
+            ksplit = -1;   // chosen by the launch from the cluster capacity
         }
     }
     if (!ksplit) ksplit = 1;
-    if (rows < 8 || rows > kBlockN || rows % 8) return LOWBIT_ERR_UNSUPPORTED;
+    if (rows < 8 || rows > kBlockN || rows % 8) return LOWBIT_ERR_UNSUPPORTED;   // (ksplit -1: automatic)
     switch (g.bits * 1000 + g.group_size) {
         case 1064: return launch_bits_gs<1, 64>(g, bt, rows, ksplit, stream);
         case 1128: return launch_bits_gs<1, 128>(g, bt, rows, ksplit, stream);
