@@ -39,6 +39,34 @@ DEFAULT_WORKLOAD = "klein_step_chain_1024sq_ternary_g128"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+def kernel_source_hash():
+    """sha256 over the CUDA sources and the ABI header: identifies the kernels a capture measured."""
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "bit_weight_only_w2_b200", "csrc")
+    inc = os.path.join(ROOT, "include")
+    files = sorted(os.path.join(csrc, f) for f in os.listdir(csrc) if f.endswith((".cu", ".cuh", ".h")))
+    files += sorted(os.path.join(inc, f) for f in os.listdir(inc) if f.endswith(".h"))
+    for f in files:
+        h.update(os.path.basename(f).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def measured_traffic(key):
+    """DRAM bytes per launch from the committed ncu summary for this workload, or None if there is
+    none or the kernels have changed since it was captured."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            entry = json.load(f).get(key)
+    except Exception:
+        return None
+    if not entry or entry.get("source_sha256") != kernel_source_hash():
+        return None
+    return entry.get("dram_bytes_per_launch")
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -381,11 +409,12 @@ def run_lowbit(args, specs, workload):
                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_steps}
 
     long_step = ms_step >= 5.0
+    traffic = measured_traffic(workload)
     if hbm_bound:
         peak_bw = peaks.get("hbm_gbs")
         achieved = launch_bytes / (launch_ms * 1e-3) / 1e9
         roofline = {"bound": "hbm", "achieved": achieved, "peak": peak_bw, "unit": "GB/s",
-                    "frac": achieved / peak_bw, "traffic": None,
+                    "frac": achieved / peak_bw, "traffic": traffic,
                     "peak_source": f"{peak_src} HBM copy bandwidth", "kernel": "lowbit_smallm_kernel",
                     "launches_timed": len(per), "algorithmic_mb_per_launch": launch_bytes / 1e6,
                     "algorithmic_gflop_per_launch": launch_flops / 1e9,
@@ -395,7 +424,7 @@ def run_lowbit(args, specs, workload):
         peak_tf = peaks.get("bf16_tflops_sustained" if long_step else "bf16_tflops")
         achieved = launch_flops / (launch_ms * 1e-3) / 1e12
         roofline = {"bound": "tensor", "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
-                    "frac": achieved / peak_tf, "traffic": None,
+                    "frac": achieved / peak_tf, "traffic": traffic,
                     "peak_source": f"{peak_src} {'sustained' if long_step else 'burst'} bf16 dense",
                     "kernel": "lowbit_gemm_kernel", "launches_timed": len(per),
                     "algorithmic_gflop_per_launch": launch_flops / 1e9,
@@ -448,9 +477,14 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--per-shape", action="store_true", help="print per-shape launch times to stderr")
+    ap.add_argument("--only-linear", default="", help="comma-separated indices of the workload's linears to run "
+                                                      "(profiling one shape); default all")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)   # at least 3 untimed warm-up steps
     specs = synth.WORKLOADS[args.workload]
+    if args.only_linear:
+        specs = [specs[int(i)] for i in args.only_linear.split(",")]
+        args.workload = f"{args.workload}[{args.only_linear}]"
     if args.impl == "reference":
         return run_reference(args, specs, args.workload)
     return run_lowbit(args, specs, args.workload)
