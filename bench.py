@@ -426,7 +426,8 @@ def run_lowbit(args, specs, workload):
         roofline = {"bound": "tensor", "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
                     "frac": achieved / peak_tf, "traffic": traffic,
                     "peak_source": f"{peak_src} {'sustained' if long_step else 'burst'} bf16 dense",
-                    "kernel": "lowbit_gemm_kernel", "launches_timed": len(per),
+                    "kernel": "lowbit_gemm_kernel (each timed launch is one lowbit_gemm call: X conversion "
+                              "pass + GEMM kernel)", "launches_timed": len(per),
                     "algorithmic_gflop_per_launch": launch_flops / 1e9,
                     "algorithmic_mb_per_launch": launch_bytes / 1e6,
                     "frac_of_burst_peak": achieved / peaks.get("bf16_tflops", peak_tf)}
