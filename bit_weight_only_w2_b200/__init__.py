@@ -128,6 +128,12 @@ def workspace_size(M: int, K: int) -> int:
     return int(load().lowbit_gemm_workspace_size(M, K))
 
 
+def _workspace_size_fast(M: int, K: int) -> int:
+    # the closed form lowbit_gemm_workspace_size returns (fp16 X copy + fp32 row factors, each
+    # rounded up to 256 bytes); tests check the two agree
+    return ((M * K * 2 + 255) // 256 + (M * 4 + 255) // 256) * 256
+
+
 _workspaces = {}
 
 
@@ -159,18 +165,29 @@ def gemm(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, zeros: Opt
         out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
     else:
         _need(out, torch.bfloat16, "out")
-    with torch.cuda.device(x.device):
-        lib = load()
-        need = workspace_size(M, K)
-        if ws is None:
-            ws = workspace(x.device, need)
-        if tile_tokens or ksplit or tile_rows:
-            st = lib.lowbit_gemm_ex(M, N, K, bits, group_size, _ptr(x), _ptr(packed), _ptr(scales), _ptr(zeros),
-                                    _ptr(out), _ptr(ws), ws.numel(), tile_tokens, tile_rows, ksplit, _stream(x))
-        else:
-            st = lib.lowbit_gemm(M, N, K, bits, group_size, _ptr(x), _ptr(packed), _ptr(scales), _ptr(zeros),
-                                 _ptr(out), _ptr(ws), ws.numel(), _stream(x))
-        _check(st, "lowbit_gemm")
+    dev = x.get_device()
+    if dev != torch.cuda.current_device():
+        with torch.cuda.device(dev):
+            return _gemm_call(x, packed, scales, zeros, bits, group_size, out, tile_tokens, ksplit, ws, tile_rows,
+                              M, N, K, dev)
+    return _gemm_call(x, packed, scales, zeros, bits, group_size, out, tile_tokens, ksplit, ws, tile_rows, M, N, K,
+                      dev)
+
+
+def _gemm_call(x, packed, scales, zeros, bits, group_size, out, tile_tokens, ksplit, ws, tile_rows, M, N, K, dev):
+    lib = _lib if _lib is not None else load()
+    if ws is None:
+        ws = workspace(x.device, _workspace_size_fast(M, K))
+    stream = torch.cuda.current_stream().cuda_stream
+    zp = None if zeros is None else zeros.data_ptr()
+    if tile_tokens or ksplit or tile_rows:
+        st = lib.lowbit_gemm_ex(M, N, K, bits, group_size, x.data_ptr(), packed.data_ptr(), scales.data_ptr(), zp,
+                                out.data_ptr(), ws.data_ptr(), ws.numel(), tile_tokens, tile_rows, ksplit, stream)
+    else:
+        st = lib.lowbit_gemm(M, N, K, bits, group_size, x.data_ptr(), packed.data_ptr(), scales.data_ptr(), zp,
+                             out.data_ptr(), ws.data_ptr(), ws.numel(), stream)
+    if st != 0:
+        raise LowbitError(st, "lowbit_gemm")
     return out
 
 

@@ -640,6 +640,9 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w, float scale) {
 
 constexpr int kConvThreads = 256;
 
+// One CTA per row of X. PER > 0: the row is held in registers (PER 16-byte chunks per thread,
+// K <= 2048 * PER), so X is read from memory once; PER == 0: any K, the row is read twice.
+template <int PER>
 __global__ void __launch_bounds__(kConvThreads) convert_x_kernel(const uint4* __restrict__ X, int K8,
                                                                  uint4* __restrict__ Xh, float* __restrict__ rowmul) {
     grid_dependency_wait();
@@ -648,7 +651,18 @@ __global__ void __launch_bounds__(kConvThreads) convert_x_kernel(const uint4* __
     const uint4* src = X + static_cast<size_t>(row) * K8;
     uint4* dst = Xh + static_cast<size_t>(row) * K8;
     uint32_t mx = 0;
-    for (int i = threadIdx.x; i < K8; i += kConvThreads) mx = absmax_bf16x8(src[i], mx);
+    uint4 v[PER > 0 ? PER : 1];
+    if (PER > 0) {
+#pragma unroll
+        for (int j = 0; j < PER; ++j) {
+            const int i = threadIdx.x + j * kConvThreads;
+            v[j] = i < K8 ? ldg_nc_v4(src + i) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int j = 0; j < PER; ++j) mx = absmax_bf16x8(v[j], mx);
+    } else {
+        for (int i = threadIdx.x; i < K8; i += kConvThreads) mx = absmax_bf16x8(src[i], mx);
+    }
     mx = __reduce_max_sync(0xffffffffu, mx);
     __shared__ uint32_t warp_max[kConvThreads / 32];
     if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = mx;
@@ -660,14 +674,22 @@ __global__ void __launch_bounds__(kConvThreads) convert_x_kernel(const uint4* __
     int e = (mx == 0 || E >= 255) ? 0 : E - 142;          // largest |x| * 2^-e in [2^15, 2^16)
     e = max(-100, min(112, e));
     const float scale = __int_as_float((127 - e) << 23);  // 2^-e
-    for (int i = threadIdx.x; i < K8; i += kConvThreads) {
-        const uint4 v = src[i];
+    auto cvt = [&](const uint4& a) {
         uint4 o;
-        o.x = bf16x2_to_f16x2(v.x, scale);
-        o.y = bf16x2_to_f16x2(v.y, scale);
-        o.z = bf16x2_to_f16x2(v.z, scale);
-        o.w = bf16x2_to_f16x2(v.w, scale);
-        dst[i] = o;
+        o.x = bf16x2_to_f16x2(a.x, scale);
+        o.y = bf16x2_to_f16x2(a.y, scale);
+        o.z = bf16x2_to_f16x2(a.z, scale);
+        o.w = bf16x2_to_f16x2(a.w, scale);
+        return o;
+    };
+    if (PER > 0) {
+#pragma unroll
+        for (int j = 0; j < PER; ++j) {
+            const int i = threadIdx.x + j * kConvThreads;
+            if (i < K8) dst[i] = cvt(v[j]);
+        }
+    } else {
+        for (int i = threadIdx.x; i < K8; i += kConvThreads) dst[i] = cvt(src[i]);
     }
     if (threadIdx.x == 0) rowmul[row] = __int_as_float((127 + e) << 23);   // 2^e
 }
@@ -683,10 +705,16 @@ lowbit_status launch_convert_x(const GemmProblem& g, cudaStream_t stream) {
     ccfg.stream = stream;
     ccfg.attrs = cattr;
     ccfg.numAttrs = 1;
-    const cudaError_t e = cudaLaunchKernelEx(
-        &ccfg, convert_x_kernel, static_cast<const uint4*>(g.X), static_cast<int>(g.K / 8),
-        static_cast<uint4*>(g.workspace),
-        reinterpret_cast<float*>(static_cast<uint8_t*>(g.workspace) + ws.rowmul_offset));
+    const int K8 = static_cast<int>(g.K / 8);
+    const uint4* x = static_cast<const uint4*>(g.X);
+    uint4* xh = static_cast<uint4*>(g.workspace);
+    float* rm = reinterpret_cast<float*>(static_cast<uint8_t*>(g.workspace) + ws.rowmul_offset);
+    cudaError_t e;
+    if (K8 <= kConvThreads) e = cudaLaunchKernelEx(&ccfg, convert_x_kernel<1>, x, K8, xh, rm);
+    else if (K8 <= 2 * kConvThreads) e = cudaLaunchKernelEx(&ccfg, convert_x_kernel<2>, x, K8, xh, rm);
+    else if (K8 <= 4 * kConvThreads) e = cudaLaunchKernelEx(&ccfg, convert_x_kernel<4>, x, K8, xh, rm);
+    else if (K8 <= 8 * kConvThreads) e = cudaLaunchKernelEx(&ccfg, convert_x_kernel<8>, x, K8, xh, rm);
+    else e = cudaLaunchKernelEx(&ccfg, convert_x_kernel<0>, x, K8, xh, rm);
     return e == cudaSuccess ? LOWBIT_OK : LOWBIT_ERR_CUDA;
 }
 
@@ -714,6 +742,76 @@ lowbit_status selftest_bounded_wait(long long limit_cycles, cudaStream_t stream)
 // ---------------------------------------------------------------------------------------------
 namespace {
 
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn();
+
+// Tensor maps are a pure function of their arguments (address, geometry, box, swizzle), so
+// encoded maps are kept in a small direct-mapped cache: a linear called again with the same
+// buffers skips the driver's encode.
+struct MapKey {
+    uint64_t base;
+    uint64_t dims[3];
+    uint64_t strides[2];
+    uint32_t box[3];
+    int dtype, rank, swz;
+    bool operator==(const MapKey& o) const {
+        return base == o.base && dims[0] == o.dims[0] && dims[1] == o.dims[1] && dims[2] == o.dims[2] &&
+               strides[0] == o.strides[0] && strides[1] == o.strides[1] && box[0] == o.box[0] &&
+               box[1] == o.box[1] && box[2] == o.box[2] && dtype == o.dtype && rank == o.rank && swz == o.swz;
+    }
+};
+
+bool encode_cached(CUtensorMap* map, CUtensorMapDataType dtype, int rank, const void* base, const uint64_t* dims,
+                   const uint64_t* strides, const uint32_t* box, CUtensorMapSwizzle swz) {
+    constexpr int kSlots = 1024;
+    struct Slot {
+        bool used;
+        MapKey key;
+        CUtensorMap map;
+    };
+    static Slot* slots = new Slot[kSlots]();
+    static std::mutex mu;
+    MapKey k = {};
+    k.base = reinterpret_cast<uint64_t>(base);
+    for (int i = 0; i < rank; ++i) {
+        k.dims[i] = dims[i];
+        k.box[i] = box[i];
+    }
+    for (int i = 0; i + 1 < rank; ++i) k.strides[i] = strides[i];
+    k.dtype = static_cast<int>(dtype);
+    k.rank = rank;
+    k.swz = static_cast<int>(swz);
+    uint64_t h = k.base * 0x9E3779B97F4A7C15ull;
+    for (int i = 0; i < 3; ++i) h ^= (k.dims[i] + 0x632BE59BD9B4E019ull * (k.box[i] + 1)) * (2 * i + 3);
+    h ^= (k.strides[0] * 31 + k.strides[1]) ^ (static_cast<uint64_t>(k.dtype) << 40) ^
+         (static_cast<uint64_t>(k.swz) << 48) ^ (static_cast<uint64_t>(rank) << 56);
+    h ^= h >> 29;
+    Slot& sl = slots[h % kSlots];
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (sl.used && sl.key == k) {
+            *map = sl.map;
+            return true;
+        }
+    }
+    auto fn = get_encode_fn();
+    if (!fn) return false;
+    cuuint64_t d[3], st[2];
+    cuuint32_t b[3], estr[3] = {1, 1, 1};
+    for (int i = 0; i < rank; ++i) {
+        d[i] = dims[i];
+        b[i] = box[i];
+    }
+    for (int i = 0; i + 1 < rank; ++i) st[i] = strides[i];
+    const CUresult r = fn(map, dtype, rank, const_cast<void*>(base), d, st, b, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return false;
+    std::lock_guard<std::mutex> lock(mu);
+    sl.used = true;
+    sl.key = k;
+    sl.map = *map;
+    return true;
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     static bool tried = false;
@@ -731,46 +829,27 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
 // X as a 3-D tensor (64 k, M rows, K/64 k-atoms) so that one box covers a whole 128-wide k-block
 // of BT token rows in the 128-byte-swizzled layout [k half][row][64 k] the MMA reads.
 bool make_map_x3d(CUtensorMap* map, const void* base, uint64_t M, uint64_t K, uint32_t box_rows) {
-    auto fn = get_encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[3] = {64, M, K / 64};
-    cuuint64_t strides[2] = {K * 2, 128};
-    cuuint32_t box[3] = {64, box_rows, 2};
-    cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
+    const uint64_t dims[3] = {64, M, K / 64};
+    const uint64_t strides[2] = {K * 2, 128};
+    const uint32_t box[3] = {64, box_rows, 2};
+    return encode_cached(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 }  // namespace
 
 bool make_map_3d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, const uint64_t (&dims)[3],
                  const uint64_t (&strides)[2], const uint32_t (&box)[3], CUtensorMapSwizzle swz) {
-    auto fn = get_encode_fn();
-    if (!fn) return false;
-    cuuint64_t d[3] = {dims[0], dims[1], dims[2]};
-    cuuint64_t st[2] = {strides[0], strides[1]};
-    cuuint32_t b[3] = {box[0], box[1], box[2]};
-    cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = fn(map, dtype, 3, const_cast<void*>(base), d, st, b, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
+    return encode_cached(map, dtype, 3, base, dims, strides, box, swz);
 }
 
 bool make_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, int elem_bytes, const void* base, uint64_t inner,
                  uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
                  CUtensorMapSwizzle swz) {
-    auto fn = get_encode_fn();
-    if (!fn) return false;
     (void)elem_bytes;
-    cuuint64_t dims[2] = {inner, outer};
-    cuuint64_t strides[1] = {row_bytes};
-    cuuint32_t box[2] = {box_inner, box_outer};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                    swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
+    const uint64_t dims[2] = {inner, outer};
+    const uint64_t strides[1] = {row_bytes};
+    const uint32_t box[2] = {box_inner, box_outer};
+    return encode_cached(map, dtype, 2, base, dims, strides, box, swz);
 }
 
 int cluster_capacity(const void* kernel, int ks, int threads, int smem_bytes) {

@@ -4,6 +4,7 @@
 
 #include <cstdint>
 #include <cstdlib>
+#include <atomic>
 #include <mutex>
 
 #include "lowbit_internal.h"
@@ -33,13 +34,20 @@ lowbit_status check_pack_args(const void* a, const void* b, int64_t N, int64_t K
 lowbit_status check_device() {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return LOWBIT_ERR_CUDA;
+    // the answer per device never changes: 1 = supported, 2 = not (0 = not yet asked)
+    static std::atomic<int> known[64];
+    if (dev >= 0 && dev < 64) {
+        const int k = known[dev].load(std::memory_order_relaxed);
+        if (k) return k == 1 ? LOWBIT_OK : LOWBIT_ERR_UNSUPPORTED_DEVICE;
+    }
     int major = 0, minor = 0;
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
         return LOWBIT_ERR_CUDA;
     // The kernels are built for sm_100a only (tcgen05 / tensor memory).
-    if (major != 10 || minor != 0) return LOWBIT_ERR_UNSUPPORTED_DEVICE;
-    return LOWBIT_OK;
+    const bool ok = major == 10 && minor == 0;
+    if (dev >= 0 && dev < 64) known[dev].store(ok ? 1 : 2, std::memory_order_relaxed);
+    return ok ? LOWBIT_OK : LOWBIT_ERR_UNSUPPORTED_DEVICE;
 }
 
 lowbit_status validate_gemm(const GemmProblem& g) {

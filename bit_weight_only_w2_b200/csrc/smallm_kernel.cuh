@@ -280,17 +280,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (x) tma_load_3d(&map_x, &full[s], st, 0, 0, kk / 64);
     };
     // The codes, scales and zeros are not written by earlier kernels of the stream that this one
-    // may overlap: thread 0 fetches the first ring's share at once, while lane 0 of warp 1 waits
-    // for those kernels and then adds X, so step 0's X is queued right behind its codes.
+    // may overlap, X may be: thread 0 queues step 0's codes, waits for those kernels, then X of
+    // step 0 and the other steps of the first ring, so step 0 is complete as early as possible
+    // (the copy engine serves requests in order).
     const int pre = min(S, total);
     if (threadIdx.x == 0) {
+        if (pre > 0) issue(0, true, false);
+        grid_dependency_wait();
         for (int gs = 0; gs < pre; ++gs) {
-            issue(gs, true, false);
+            if (gs > 0) issue(gs, true, false);
+            issue(gs, false, true);
             iss[gs] = 1;
         }
-    } else if (threadIdx.x == 32) {
-        grid_dependency_wait();
-        for (int gs = 0; gs < pre; ++gs) issue(gs, false, true);
     }
 
     const int w = warp;
@@ -440,33 +441,41 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
 
-        // ---- tile end: sum the eight warps' partials in a fixed order: (w + (w + 4)) for
-        // w < 4, then ((0 + 1) + 2) + 3.
+        // ---- tile end: sum the eight warps' partials in a fixed order. On a CTA's only tile the
+        // drained ring holds all eight: one exchange, ((((w0 + w1) + w2) + ...) + w7). Otherwise
+        // the ring already holds the next tile's steps and `red` takes two rounds:
+        // (w + (w + 4)) for w < 4, then ((0 + 1) + 2) + 3.
         grid_dependency_wait();   // Y may still be read by the kernel this one overlaps
-        cta_bar();                // the previous tile's readers of `red` are done
-        if (w >= 4) {
+        const bool one_round = my_tiles == 1 && static_cast<uint32_t>(S) * p.stage_bytes >= kWarps * NOCT * 512u;
+        float4* rbuf = one_round ? reinterpret_cast<float4*>(ring) : red;
+        const int nslot = one_round ? kWarps : 4;
+        cta_bar();                // the ring is drained / the previous tile's readers of `red` are done
+        if (one_round || w >= 4) {
+            const int slot = one_round ? w : w - 4;
 #pragma unroll
             for (int o = 0; o < NOCT; ++o)
-                red[((w - 4) * NOCT + o) * 32 + lane] = make_float4(acc[o][0], acc[o][1], acc[o][2], acc[o][3]);
+                rbuf[(slot * NOCT + o) * 32 + lane] = make_float4(acc[o][0], acc[o][1], acc[o][2], acc[o][3]);
         }
         cta_bar();
-        if (w < 4) {
+        if (!one_round) {
+            if (w < 4) {
 #pragma unroll
-            for (int o = 0; o < NOCT; ++o) {
-                const float4 v = red[(w * NOCT + o) * 32 + lane];
-                acc[o][0] += v.x;
-                acc[o][1] += v.y;
-                acc[o][2] += v.z;
-                acc[o][3] += v.w;
+                for (int o = 0; o < NOCT; ++o) {
+                    const float4 v = red[(w * NOCT + o) * 32 + lane];
+                    acc[o][0] += v.x;
+                    acc[o][1] += v.y;
+                    acc[o][2] += v.z;
+                    acc[o][3] += v.w;
+                }
             }
-        }
-        cta_bar();
-        if (w < 4) {
+            cta_bar();
+            if (w < 4) {
 #pragma unroll
-            for (int o = 0; o < NOCT; ++o)
-                red[(w * NOCT + o) * 32 + lane] = make_float4(acc[o][0], acc[o][1], acc[o][2], acc[o][3]);
+                for (int o = 0; o < NOCT; ++o)
+                    red[(w * NOCT + o) * 32 + lane] = make_float4(acc[o][0], acc[o][1], acc[o][2], acc[o][3]);
+            }
+            cta_bar();
         }
-        cta_bar();
 #pragma unroll
         for (int o = 0; o < NOCT; ++o) acc[o][0] = acc[o][1] = acc[o][2] = acc[o][3] = 0.f;
 
@@ -483,10 +492,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         };
         auto tile_sum = [&](int o) {
-            float4 v = red[o * 32 + lane];
+            float4 v = rbuf[o * 32 + lane];
 #pragma unroll
-            for (int r = 1; r < 4; ++r) {
-                const float4 u = red[(r * NOCT + o) * 32 + lane];
+            for (int r = 1; r < kWarps; ++r) {
+                if (r >= nslot) break;
+                const float4 u = rbuf[(r * NOCT + o) * 32 + lane];
                 v.x += u.x;
                 v.y += u.y;
                 v.z += u.z;

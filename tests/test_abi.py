@@ -117,3 +117,10 @@ def test_pack_rejects_before_launch(lib):
     assert lib.lowbit_pack(A, 4, 64, 3, A, None) == 1
     assert lib.lowbit_pack(A + 1, 4, 64, 2, A, None) == 2
     assert lib.lowbit_unpack(None, 4, 64, 2, A, None) == 1
+
+
+def test_binding_workspace_size_matches_library():
+    """The Python binding's closed-form workspace size equals lowbit_gemm_workspace_size."""
+    import bit_weight_only_w2_b200 as lb
+    for M, K in [(1, 64), (16, 2560), (512, 9728), (4608, 12288), (7, 192), (0, 64), (3, 128)]:
+        assert lb._workspace_size_fast(M, K) == lb.workspace_size(M, K), (M, K)
