@@ -67,6 +67,36 @@ def measured_traffic(key):
     return entry.get("dram_bytes_per_launch")
 
 
+def rotation_copies(step_bytes_: int, weight_bytes_: int, l2_bytes: int) -> int:
+    """Distinct weight copies a workload rotates through: 1 if its bytes reach twice L2, else at
+    least 20 and enough that the copies' weights exceed 2.2x L2 (at most 256)."""
+    if step_bytes_ >= 2 * l2_bytes:
+        return 1
+    return min(256, max(20, -(-int(2.2 * l2_bytes) // max(1, weight_bytes_))))
+
+
+def is_hbm_bound(flops: float, nbytes: float, peaks: dict) -> bool:
+    """Below the ridge point (peak flop/s over peak byte/s) a workload is bound by HBM."""
+    ridge = peaks.get("bf16_tflops", 1590.0) * 1e12 / (peaks.get("hbm_gbs", 6650.0) * 1e9)
+    return flops / nbytes < ridge
+
+
+def max_over_ranks(v: float, world: int, device=None) -> float:
+    """The maximum of v over all ranks of the default process group (v itself when alone)."""
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(world: int, flops_per_step: float, ms_per_step: float) -> float:
+    """Whole-job TFLOP/s: every rank runs the step (replicas), timed by the slowest rank."""
+    return world * flops_per_step / (ms_per_step * 1e-3) / 1e12
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -273,28 +303,21 @@ def run_lowbit(args, specs, workload):
     l2_bytes = torch.cuda.get_device_properties(device).L2_cache_size
     # A workload that fits in L2 rotates distinct copies of its weights (at least 20, and enough
     # to exceed twice L2) so that every step reads them from HBM, with no flush between steps.
-    copies = 1
-    if nbytes < 2 * l2_bytes:
-        copies = min(256, max(20, -(-int(2.2 * l2_bytes) // max(1, weight_bytes(specs)))))
+    copies = rotation_copies(nbytes, weight_bytes(specs), l2_bytes)
     items, desc_sets = setup(specs, device, lb, torch, pinned=not args.no_e2e, copies=copies)
     descs = desc_sets[0]
     stream = torch.cuda.current_stream(device)
     peaks, peak_src = load_peaks()
     # bound of the workload: below the ridge point (peak flop/s per peak byte/s) it is HBM-bound
-    ridge = peaks.get("bf16_tflops", 1590.0) * 1e12 / (peaks.get("hbm_gbs", 6650.0) * 1e9)
-    hbm_bound = flops / nbytes < ridge
+    hbm_bound = is_hbm_bound(flops, nbytes, peaks)
     launches_per_step = sum(1 if s.M <= 16 else 2 for s in specs)   # X conversion + GEMM above 16 tokens
 
     def barrier():
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(v):
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def ranks_max(v):
+        return max_over_ranks(v, world, device)
 
     # Each step is one lowbit_gemm_batch over the workload's linears, captured once per weight
     # copy as a CUDA graph and replayed, so the timed region measures the GPU rather than the
@@ -337,9 +360,9 @@ def run_lowbit(args, specs, workload):
     ms_total = a.elapsed_time(b)
     barrier()
     clk = clocks.stop()
-    ms_total = max_over_ranks(ms_total)
+    ms_total = ranks_max(ms_total)
     ms_step = ms_total / args.steps
-    value = world * flops / (ms_step * 1e-3) / 1e12
+    value = job_value(world, flops, ms_step)
     if lb.device_status() != 0:
         raise RuntimeError("kernel timeout reported during the timed steps")
 
@@ -404,7 +427,7 @@ def run_lowbit(args, specs, workload):
                 it["y_host"].copy_(it["y"], non_blocking=True)
         b.record(stream)
         torch.cuda.synchronize(device)
-        e2e_ms = max_over_ranks(a.elapsed_time(b)) / e2e_steps
+        e2e_ms = ranks_max(a.elapsed_time(b)) / e2e_steps
         e2e = {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_steps}
 
