@@ -111,7 +111,10 @@ lowbit_status lowbit_gemm(int64_t M, int64_t N, int64_t K, int bits, int group_s
  * tuning and tests (each 0 = automatic):
  *   tile_tokens  tokens per CTA tile of the tensor-memory kernel: 16, 32, 64, 128 or 256; or 1
  *                for the small-M kernel on warp-level MMAs (M <= 16 only; chosen automatically
- *                for M <= 16; it reads X directly and leaves the workspace untouched)
+ *                for M <= 16; it reads X directly and leaves the workspace untouched). That
+ *                kernel sums unscaled codes times X in fp32 per group before applying the
+ *                scale, so its results are exact only for |x| below about 2^114; the
+ *                tensor-memory kernel (M > 16, or tile_tokens >= 16) covers the full bf16 range
  *   tile_rows    weight rows per CTA tile: a multiple of 8 up to 128 (128 unless the shape is
  *                small; fewer rows give more CTAs, each streaming the whole K)
  *   ksplit       number of K slices summed across a thread-block cluster, 1..8 (1 = no split;

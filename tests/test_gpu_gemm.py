@@ -222,7 +222,8 @@ FULL = [s for w in ("qkv_512sq_ternary_g128", "mlp_1024sq_binary_g128", "te_m512
 
 @pytest.mark.parametrize("spec", FULL, ids=lambda s: s.name)
 def test_full_size_sampled(spec):
-    sampled_check(spec)
+    worst = sampled_check(spec)
+    print(f"\n{spec.name} M={spec.M} K={spec.K} N={spec.N}: max err/bound {worst:.3f}")
 
 
 def chain_distinct():
@@ -234,7 +235,8 @@ def chain_distinct():
 
 @pytest.mark.parametrize("spec", chain_distinct(), ids=lambda s: s.name)
 def test_chain_shapes_sampled(spec):
-    sampled_check(spec, n_random=2048, n_rows=4, n_cols=4)
+    worst = sampled_check(spec, n_random=2048, n_rows=4, n_cols=4)
+    print(f"\n{spec.name} M={spec.M} K={spec.K} N={spec.N}: max err/bound {worst:.3f}")
 
 
 def test_batch_matches_single_calls():
@@ -300,3 +302,28 @@ def test_extreme_row_magnitudes():
         if m == 2:
             continue
         _gpu.check_close(y[m], ref[m], what=f"row {m}")
+
+
+@pytest.mark.parametrize("bits,gs", [(1, 128), (2, 128), (4, 64)])
+def test_small_m_row_magnitudes(bits, gs):
+    """The small-M kernel sums unscaled codes times X in fp32 per group, so it is exact for
+    |x| up to about 2^114; rows scaled by 2^100 and 2^-100, tiny and zero rows match the oracle
+    row by row."""
+    spec = spec_for(bits, gs, 9, 1024, 264, seed=41)
+    prob = synth.make_problem(spec)
+    x = _pins.x_as_f64(prob.x_bf16)
+    x[0] *= 2.0 ** 100
+    x[1] *= 2.0 ** -60
+    x[2] = 0.0
+    x[3] *= 2.0 ** -100
+    x[4, 5] = 1.5 * 2.0 ** 104          # one huge entry in an otherwise ordinary row
+    prob.x_bf16 = _pins.bf16_bits_from_f32(x.astype(np.float32))
+    ref = oracle.gemm(prob.x_bf16, _gpu.oracle_packed(prob), prob.scales, prob.zeros, spec.N, bits, gs)
+    xd, packed, s, z = _gpu.dev_problem(prob)
+    y = _gpu.y_to_f64(lb.gemm(xd, packed, s, z, bits, gs, tile_tokens=1))
+    torch.cuda.synchronize()
+    assert np.all(y[2] == 0.0)
+    for m in range(spec.M):
+        if m == 2:
+            continue
+        _gpu.check_close(y[m:m + 1], ref[m:m + 1], what=f"row {m}")
