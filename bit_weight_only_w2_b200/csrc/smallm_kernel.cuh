@@ -150,50 +150,11 @@ __device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t* p, uint32_t v) {
     return old;
 }
 
-// Makes this thread's prior writes (and, through the preceding CTA barrier, its CTA's) visible
-// at cluster scope before the relaxed arrivals that follow it.
-__device__ __forceinline__ void fence_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
-
-// Arrive on the barrier at `cluster_addr` (a shared::cluster address) without ordering; pair
-// with fence_cluster().
-__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_addr) {
-    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
-}
 
 __device__ __forceinline__ void st_shared_cluster_v4(uint32_t addr, float4 v) {
     asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.x), "f"(v.y), "f"(v.z),
                  "f"(v.w)
                  : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait_acq_cluster(uint64_t* bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}\n"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-// Bounded wait with cluster-scope acquire (for barriers other CTAs of the cluster arrive on).
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                                  unsigned* status_word) {
-    const long long t0 = clock64();
-    uint32_t it = 0;
-    while (!mbar_try_wait_acq_cluster(bar, parity)) {
-        if ((++it & 63u) == 0) {
-            if (*abort_flag) return false;
-            if (clock64() - t0 > kWaitLimitCycles) {
-                atomicOr(status_word, kDevErrTimeout);
-                *abort_flag = 1;
-                return false;
-            }
-        }
-    }
-    return true;
 }
 
 // Exact bf16 pairs of two neighbouring codes (k, k + 1) at pair index c of a packed word.
@@ -231,9 +192,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     float4* red = reinterpret_cast<float4*>(smem + p.red_off);
     float4* part = reinterpret_cast<float4*>(smem + p.part_off);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + p.bar_off);
-    uint64_t* pready = full + kMaxStages;      // every rank's part of the tile is written
-    uint64_t* pfree = pready + 1;              // every rank has read this CTA's part
-    uint32_t* cnt = reinterpret_cast<uint32_t*>(pfree + 1);   // per slot: warps done, all rounds
+    uint32_t* cnt = reinterpret_cast<uint32_t*>(full + kMaxStages);   // per slot: warps done, all rounds
     uint32_t* iss = cnt + kMaxStages;                         // per slot: fills issued
     volatile int* abort_flag = reinterpret_cast<volatile int*>(iss + kMaxStages);
 
@@ -254,13 +213,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             cnt[i] = 0;
             iss[i] = 0;
         }
-        mbar_init(pready, ks);
-        mbar_init(pfree, ks);
         *abort_flag = 0;
         fence_mbar_init();
     }
     __syncthreads();
-    if (ks > 1) cluster_sync_all();   // other ranks arrive on this CTA's barriers
+    if (ks > 1) cluster_sync_all();   // every CTA of the cluster has started (remote stores target it)
     grid_launch_dependents();
 
     // Ring step `gs` of this CTA: tile blockIdx.x + (gs / nst) * gridDim.x, K step gs % nst.
@@ -281,9 +238,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     // The codes, scales and zeros are not written by earlier kernels of the stream that this one
     // may overlap, X may be: thread 0 queues step 0's codes, waits for those kernels, then X of
-    // step 0 and the other steps of the first ring, so step 0 is complete as early as possible
-    // (the copy engine serves requests in order).
-    const int pre = min(S, total);
+    // step 0 and the rest of the first ring (the copy engine serves requests in order, so step 0
+    // completes first). The ring runs `look` = S steps ahead: the last warp out of step it
+    // queues step it + look. (Measured on the 16-token text-encoder shapes: looking 2, 3 or S
+    // steps ahead gives the same time.)
+    const int look = S;
+    const int pre = min(look, total);
     if (threadIdx.x == 0) {
         if (pre > 0) issue(0, true, false);
         grid_dependency_wait();
@@ -431,12 +391,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             __syncwarp();
-            // Release the slot; the last warp out refills it with ring step it + S.
+            // Release the slot; the last warp out queues ring step it + look (into the slot of step
+            // it + look - S <= it, which every warp has left).
             if (lane == 0) {
                 const uint32_t prev = atom_add_acq_rel(&cnt[s], 1);
-                if ((prev & (kWarps - 1)) == kWarps - 1 && it + S < total && !*abort_flag) {
-                    issue(it + S, true, true);
-                    iss[s] += 1;
+                if ((prev & (kWarps - 1)) == kWarps - 1 && it + look < total && !*abort_flag) {
+                    issue(it + look, true, true);
+                    iss[(it + look) % S] += 1;
                 }
             }
         }
@@ -508,22 +469,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int o = w; o < NOCT; o += kWarps) store(o, tile_sum(o));
         } else {
             // Octet o is finished by rank o % ks: every rank stores its tile sum of o straight into
-            // that rank's receive buffer (slot [own rank][o / ks]), then the finishing rank adds
-            // the slots in rank order. pready: all ranks' sums have landed here; pfree: every
-            // finishing rank has consumed what this rank sent, so its buffers may be reused.
+            // that rank's receive buffer (slot [own rank][o / ks]); after a cluster barrier the
+            // finishing rank adds the slots in rank order; a second barrier keeps the buffers
+            // (and every CTA) alive until all ranks have read them.
             const int per = (NOCT + ks - 1) / ks;
-            if (ti > 0)
-                ok = __all_sync(0xffffffffu, mbar_wait_cluster(pfree, (ti - 1) & 1u, abort_flag, p.status)) && ok;
             for (int o = w; o < NOCT; o += kWarps) {
                 const uint32_t slot = smem_u32(part + ((rank * per + o / ks) * 32 + lane));
                 st_shared_cluster_v4(map_shared_rank(slot, o % ks), tile_sum(o));
             }
-            cta_bar();
-            if (threadIdx.x == 0) {
-                fence_cluster();
-                for (int r = 0; r < ks; ++r) mbar_arrive_cluster_relaxed(map_shared_rank(smem_u32(pready), r));
-            }
-            ok = __all_sync(0xffffffffu, mbar_wait_cluster(pready, ti & 1u, abort_flag, p.status)) && ok;
+            cluster_sync_all();
             for (int o = w; o < NOCT; o += kWarps) {
                 if (o % ks != rank) continue;
                 const int li = o / ks;
@@ -539,16 +493,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 store(o, sum);
             }
-            cta_bar();
-            if (threadIdx.x == 0) {
-                fence_cluster();
-                for (int r = 0; r < ks; ++r) mbar_arrive_cluster_relaxed(map_shared_rank(smem_u32(pfree), r));
-            }
+            cluster_sync_all();
         }
     }
-    // Stay resident until every rank has read this CTA's last partial sums, and leave no copy in
-    // flight into shared memory (only possible after an aborted wait).
-    if (ks > 1 && ti > 0) mbar_wait_cluster(pfree, (ti - 1) & 1u, abort_flag, p.status);
+    // Leave no copy in flight into shared memory (only possible after an aborted wait).
     cta_bar();
     if (threadIdx.x == 0 && *abort_flag) {
         int zero = 0;
