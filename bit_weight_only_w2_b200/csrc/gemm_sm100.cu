@@ -45,6 +45,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <mutex>
 
 #include <cstdint>
@@ -903,11 +904,15 @@ template <int BITS, int GS, int BT>
 lowbit_status launch(const GemmProblem& g, int rows, int ksplit_request, cudaStream_t stream) {
     using C = Cfg<BITS, GS, BT>;
     auto kernel = lowbit_gemm_kernel<BITS, GS, BT>;
-    static bool attr_done = false;
-    if (!attr_done) {
+    // the shared-memory opt-in is per device: one bit per device that has it
+    static std::atomic<uint64_t> attr_devices{0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return LOWBIT_ERR_CUDA;
+    const uint64_t bit = dev < 64 ? (uint64_t(1) << dev) : 0;
+    if (!bit || !(attr_devices.load(std::memory_order_acquire) & bit)) {
         if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
             return LOWBIT_ERR_CUDA;
-        attr_done = true;
+        attr_devices.fetch_or(bit, std::memory_order_acq_rel);
     }
     CUtensorMap mx, mw, ms, mz;
     const int K = static_cast<int>(g.K), N = static_cast<int>(g.N), M = static_cast<int>(g.M);

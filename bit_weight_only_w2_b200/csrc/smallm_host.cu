@@ -22,18 +22,22 @@ const void* kernel_for(int bits, int gs, int noct) {
 
 std::mutex g_mu;
 
-// Allows the kernel the full shared memory once per entry point.
+// Allows the kernel the full shared memory, once per entry point and device (the opt-in is a
+// per-device function attribute).
 bool prepare(const void* fn) {
-    static const void* done[3 * 2 * kMaxOct] = {nullptr};
+    struct Done {
+        const void* fn;
+        int dev;
+    };
+    static Done done[8 * 3 * 2 * kMaxOct];
+    static int used = 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
     std::lock_guard<std::mutex> lock(g_mu);
-    for (const void* d : done)
-        if (d == fn) return true;
+    for (int i = 0; i < used; ++i)
+        if (done[i].fn == fn && done[i].dev == dev) return true;
     if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit) != cudaSuccess) return false;
-    for (const void*& d : done)
-        if (!d) {
-            d = fn;
-            break;
-        }
+    if (used < static_cast<int>(sizeof(done) / sizeof(done[0]))) done[used++] = Done{fn, dev};
     return true;
 }
 

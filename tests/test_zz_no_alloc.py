@@ -38,7 +38,8 @@ def call_noalloc(f, spec, x, packed, s, z, y):
 def test_noalloc_matches_gemm_on_two_calls_in_a_row():
     f = noalloc_fn()
     specs = [LinearSpec("noalloc_a", 300, 512, 520, bits=2, group_size=128, p0=0.4, seed=41),
-             LinearSpec("noalloc_b", 96, 1024, 264, bits=4, group_size=64, scale_lo=0.002, scale_hi=0.01, seed=42)]
+             LinearSpec("noalloc_b", 96, 1024, 264, bits=4, group_size=64, scale_lo=0.002, scale_hi=0.01, seed=42),
+             LinearSpec("noalloc_c", 16, 2048, 1032, bits=1, group_size=128, seed=43)]   # small-M kernel
     for spec in specs:
         prob = synth.make_problem(spec)
         x, packed, s, z = _gpu.dev_problem(prob)
