@@ -110,6 +110,47 @@ def chain_linears(image_hw: int = 1024, text_tokens: int = 512, d: int = D,
     return out
 
 
+def chain_linears_separate_qkv(image_hw: int = 1024, text_tokens: int = 512, d: int = D,
+                               n_double: int = 5, n_single: int = 20) -> List[LinearSpec]:
+    """One denoise step with the transformer's unfused projection layout: each double-stream
+    block has separate image Q, K, V (d -> d each), out, MLP-up, MLP-down, and the text stream's
+    add-Q, add-K, add-V, add-out, MLP-up, MLP-down (12 linears); single-stream blocks keep their
+    fused QKV+MLP-in and out (2 linears). 5 x 12 + 20 x 2 = 100 linears (card: 100 low-bit linear
+    layers, Q/K/V and add-Q/K/V among them). Seeds and streams follow chain_linears."""
+    m_img = (image_hw // 16) * (image_hw // 16)
+    m_all = m_img + text_tokens
+    out: List[LinearSpec] = []
+    common = dict(bits=2, group_size=128, p0=0.4, scale_lo=0.005, scale_hi=0.02)
+    blk = 0
+    for _ in range(n_double):
+        slot = 0
+        for stream_name, m in (("img", m_img), ("txt", text_tokens)):
+            for lname, k, n in (("q", d, d), ("k", d, d), ("v", d, d), ("out", d, d), ("mlp_up", d, 3 * d),
+                                ("mlp_down", 3 * d, d)):
+                out.append(LinearSpec(f"double{blk}.{stream_name}.{lname}", m, k, n, seed=blk,
+                                      stream_base=100 * (slot + 1), **common))
+                slot += 1
+        blk += 1
+    for _ in range(n_single):
+        out.append(LinearSpec(f"single{blk}.qkv_mlp_in", m_all, d, 6 * d, seed=blk, stream_base=100, **common))
+        out.append(LinearSpec(f"single{blk}.out", m_all, 4 * d, d, seed=blk, stream_base=200, **common))
+        blk += 1
+    return out
+
+
+def text_encoder_mlp_layers(tokens: int, layers: int = 4) -> List[LinearSpec]:
+    """The Qwen3 text encoder's MLP linears for `layers` layers (gate and up 2560 -> 9728, down
+    9728 -> 2560; uint4, group 64 per the mlx article's component architecture). The layer count
+    is representative, not taken from the pages."""
+    common = dict(bits=4, group_size=64, scale_lo=0.002, scale_hi=0.01)
+    out: List[LinearSpec] = []
+    for layer in range(layers):
+        for j, (lname, k, n) in enumerate((("gate", TE_H, TE_I), ("up", TE_H, TE_I), ("down", TE_I, TE_H))):
+            out.append(LinearSpec(f"te{layer}.{lname}{tokens}", tokens, k, n, seed=layer,
+                                  stream_base=10 * (j + 1), **common))
+    return out
+
+
 WORKLOADS = {
     # tiny ternary, uniform codes, group 64
     "tiny_ternary_g64": [LinearSpec("tiny", 64, 256, 512, bits=2, group_size=64, p0=1.0 / 3.0)],
@@ -135,4 +176,9 @@ WORKLOADS = {
     "klein_step_chain_1024sq_ternary_g128": chain_linears(),
     # its largest linear on its own: a single-stream block's fused QKV + MLP-in (profiling case)
     "klein_single_qkv_mlp_in_1024sq_ternary_g128": [chain_linears()[40]],
+    # the same step with separate Q/K/V and add-Q/K/V projections: 100 linears
+    "klein_step_linears100_1024sq_ternary_g128": chain_linears_separate_qkv(),
+    # four text-encoder MLP layers (gate, up, down) at 512 and at 16 tokens
+    "te_mlp4_m512_uint4_g64": text_encoder_mlp_layers(512),
+    "te_mlp4_m16_uint4_g64": text_encoder_mlp_layers(16),
 }

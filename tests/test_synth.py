@@ -59,3 +59,26 @@ def test_workloads_shapes():
     for specs in synth.WORKLOADS.values():
         for s in specs:
             assert s.K % s.group_size == 0
+
+
+def test_unfused_projection_layout_has_100_linears():
+    """Separate Q/K/V and add-Q/K/V per double block: 5 x 12 + 20 x 2 = 100 linears, the same
+    work and weights as the fused layout."""
+    sep = synth.WORKLOADS["klein_step_linears100_1024sq_ternary_g128"]
+    fused = synth.chain_linears()
+    assert len(sep) == 100
+    assert sum(s.flops for s in sep) == sum(s.flops for s in fused)
+    wb = lambda specs: sum(s.N * s.K * s.bits // 8 + (s.K // s.group_size) * s.N * 2 for s in specs)  # noqa: E731
+    assert wb(sep) == wb(fused)
+    q = [s for s in sep if s.name.endswith(".q")]
+    assert len(q) == 10 and all((s.K, s.N) == (3072, 3072) for s in q)
+
+
+def test_text_encoder_layer_workloads():
+    for tokens in (512, 16):
+        specs = synth.WORKLOADS[f"te_mlp4_m{tokens}_uint4_g64"]
+        assert len(specs) == 12
+        assert all(s.M == tokens and s.bits == 4 and s.group_size == 64 for s in specs)
+        assert sorted({(s.K, s.N) for s in specs}) == [(2560, 9728), (9728, 2560)]
+        # every linear draws its own weights
+        assert len({(s.seed, s.stream_base) for s in specs}) == 12
