@@ -94,6 +94,11 @@ def test_gemm_ex_rejects_bad_tile(lib):
     assert st == 3
     st = lib.lowbit_gemm_ex(16, 128, 256, 2, 128, A, A, A, None, A, A, WS, 16, 136, 0, None)  # rows > 128
     assert st == 3
+    # the small-M kernel (tile_tokens = 1) serves at most 16 tokens
+    st = lib.lowbit_gemm_ex(17, 128, 256, 2, 128, A, A, A, None, A, A, WS, 1, 0, 0, None)
+    assert st == 3
+    st = lib.lowbit_gemm_ex(16, 128, 256, 2, 128, A, A, A, None, A, A, WS, 1, 12, 0, None)      # rows % 8
+    assert st == 3
 
 
 def test_batch_validates_all_first(lib):
