@@ -32,10 +32,15 @@
  * Bonsai-Image-Demo PR #20 describes, into uint32 words as the packed MLX checkpoint
  * of image-studio's backend.md stores them):
  *   cpw = 32 / bits codes per word; row n owns words [n * K/cpw, (n+1) * K/cpw).
- *   The code of column k lives in word j = k / cpw at offset i = k % cpw, in bits
- *   [pos, pos + bits) with pos = (i % 2) * 16 + (i / 2) * bits:
- *   even offsets fill the low 16 bits, odd offsets the high 16 bits, each half
- *   LSB-first.
+ *   Offset i of a word (0 .. cpw-1) occupies bits [pos, pos + bits) with
+ *   pos = (i % 2) * 16 + (i / 2) * bits: even offsets fill the low 16 bits, odd offsets
+ *   the high 16 bits, each half LSB-first, so the offsets 2p and 2p + 1 form pair p.
+ *   Which column an offset holds (the pages leave the order inside the packed words open):
+ *   - plain order (every binary word, and the words of a 2- or 4-bit row after its last
+ *     whole block of four): word j, offset i holds column cpw * j + i;
+ *   - block order (2- and 4-bit rows, words taken in blocks of four, so a block spans
+ *     4 * cpw columns: 32 for 4-bit, 64 for ternary): in word q (0..3) of block b, pair p
+ *     holds columns 4 * cpw * b + 8 * p + 2 * q (low half) and that + 1 (high half).
  *
  * Inputs x are bf16, scales and zeros fp16; both are passed as raw bit patterns and
  * widened to fp64 exactly (IEEE 754 binary16 / bfloat16 definitions below).
@@ -135,6 +140,29 @@ static int valid_shape(int64_t N, int64_t K, int bits) {
 
 static int bit_pos(int64_t i, int bits) { return (int)((i % 2) * 16 + (i / 2) * bits); }
 
+/* Column held at offset i of word j of a row of wpr words (the order rules above). */
+static int64_t column_of(int64_t j, int64_t i, int64_t wpr, int bits) {
+    int64_t cpw = 32 / bits;
+    if (bits != 1 && j < wpr / 4 * 4) {
+        int64_t b = j / 4, q = j % 4, p = i / 2, d = i % 2;
+        return 4 * cpw * b + 8 * p + 2 * q + d;
+    }
+    return cpw * j + i;
+}
+
+/* Word j and offset i that hold column k of a row of K columns (the inverse of column_of). */
+static void locate(int64_t k, int64_t K, int bits, int64_t* j, int64_t* i) {
+    int64_t cpw = 32 / bits, span = 4 * cpw;
+    if (bits != 1 && k < (K / cpw) / 4 * span) {
+        int64_t b = k / span, r = k % span;
+        *j = 4 * b + (r % 8) / 2;
+        *i = 2 * (r / 8) + r % 2;
+    } else {
+        *j = k / cpw;
+        *i = k % cpw;
+    }
+}
+
 /* codes [N][K] int8 -> packed [N][K*bits/32] uint32. Returns the number of invalid
  * codes (their fields are written as 0), or -1 for an invalid shape. */
 ORACLE_API int64_t oracle_pack(const int8_t* codes, int64_t N, int64_t K, int bits, uint32_t* packed) {
@@ -147,7 +175,7 @@ ORACLE_API int64_t oracle_pack(const int8_t* codes, int64_t N, int64_t K, int bi
             uint32_t w = 0;
             for (int64_t i = 0; i < cpw; ++i) {
                 uint32_t field = 0;
-                if (code_field(codes[n * K + j * cpw + i], bits, &field)) { bad++; field = 0; }
+                if (code_field(codes[n * K + column_of(j, i, words, bits)], bits, &field)) { bad++; field = 0; }
                 w |= field << bit_pos(i, bits);
             }
             packed[n * words + j] = w;
@@ -158,9 +186,10 @@ ORACLE_API int64_t oracle_pack(const int8_t* codes, int64_t N, int64_t K, int bi
 
 /* The field of weight (n, k). */
 static uint32_t field_at(const uint32_t* packed, int64_t K, int bits, int64_t n, int64_t k) {
-    int64_t cpw = 32 / bits;
-    uint32_t word = packed[n * (K / cpw) + k / cpw];
-    return (word >> bit_pos(k % cpw, bits)) & ((1u << bits) - 1u);
+    int64_t cpw = 32 / bits, j, i;
+    locate(k, K, bits, &j, &i);
+    uint32_t word = packed[n * (K / cpw) + j];
+    return (word >> bit_pos(i, bits)) & ((1u << bits) - 1u);
 }
 
 /* packed -> codes. Returns the number of invalid fields (ternary f == 3, written as 0),

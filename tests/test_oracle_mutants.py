@@ -33,8 +33,11 @@ MUTATIONS = {
                              "double s = oracle_f16_to_f64(scales[((k + 1) % K / g) * N + n]);"),
     "fp16_exponent_bias": ("v = ldexp(1024.0 + (double)f, e - 25);", "v = ldexp(1024.0 + (double)f, e - 24);"),
     "bf16_shift": ("uint32_t b = (uint32_t)h << 16;", "uint32_t b = (uint32_t)h << 15;"),
-    "word_row_stride": ("uint32_t word = packed[n * (K / cpw) + k / cpw];",
-                        "uint32_t word = packed[n * (K / cpw) + (k / cpw) % 1];"),
+    "word_row_stride": ("uint32_t word = packed[n * (K / cpw) + j];",
+                        "uint32_t word = packed[n * (K / cpw) + j % 1];"),
+    "block_pair_and_lane_swapped": ("return 4 * cpw * b + 8 * p + 2 * q + d;",
+                                    "return 4 * cpw * b + 8 * q + 2 * p + d;"),
+    "block_order_not_used": ("if (bits != 1 && j < wpr / 4 * 4) {", "if (bits != 1 && j < 0) {"),
     "ternary_field_map": ("if (c >= -1 && c <= 1) { *field = (uint32_t)(c + 1); return 0; }",
                           "if (c >= -1 && c <= 1) { *field = (uint32_t)(c + 1) ^ 2u; return 0; }"),
 }
