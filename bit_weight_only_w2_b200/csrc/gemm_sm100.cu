@@ -141,7 +141,10 @@ struct KernelParams {
 };
 
 // ---------------------------------------------------------------------------------------------
-// Decoders: one 64-wide K half of one weight row -> 32 fp16x2 values (even k low, odd k high).
+// Decoders: one 64-wide K half of one weight row -> 32 fp16x2 values (even k low, odd k high),
+// out[i] holding columns 2i and 2i + 1 of the half. 2- and 4-bit words are in block order
+// (word q of a four-word block holds, in pair p, columns 8p + 2q and 8p + 2q + 1 of the
+// block), so pair p of word w lands in out[4p + q] of its block; binary words are in plain order.
 // ---------------------------------------------------------------------------------------------
 
 // Binary: bit 1 -> +s, 0 -> -s. Pair c of a word is (bit c, bit 16 + c); shifting the word
@@ -159,7 +162,8 @@ __device__ __forceinline__ void decode_half_b1(uint32_t w0, uint32_t w1, uint32_
 // field inside the 10-bit mantissa). One fp16x2 FMA computes e * 4^-j - (1024 * 4^-j + 1) =
 // f - 1 = t exactly (the exact result is representable, so nothing rounds) and a multiply by
 // s gives t * s exactly. Pairs 0..4 are decoded in place, pairs 5..7 after one shift by 10.
-__device__ __forceinline__ void decode_word_b2(uint32_t v, uint32_t s2, uint32_t* out) {
+// Word q of the half's only block: pair c goes to out[4c + q].
+__device__ __forceinline__ void decode_word_b2(uint32_t v, uint32_t s2, uint32_t* out, int q) {
     constexpr uint32_t kMagic = 0x64006400u;                                           // 1024.0
     constexpr uint32_t kMul[5] = {0x3C003C00u, 0x34003400u, 0x2C002C00u, 0x24002400u, 0x1C001C00u};  // 4^-j
     constexpr uint32_t kAdd[5] = {0xE401E401u, 0xDC04DC04u, 0xD410D410u, 0xCC40CC40u, 0xC500C500u};  // -(1024*4^-j+1)
@@ -169,14 +173,15 @@ __device__ __forceinline__ void decode_word_b2(uint32_t v, uint32_t s2, uint32_t
         const int j = (c < 5) ? c : c - 5;
         const uint32_t e = and_or(v >> shift, 0x00030003u << (2 * j), kMagic);
         const uint32_t t = f16x2_fma(e, kMul[j], kAdd[j]);
-        out[c] = f16x2_mul(t, s2);
+        out[4 * c + q] = f16x2_mul(t, s2);
     }
 }
 
 // uint4: the nibbles of a pair, left at bit 4j of each half (j <= 1), OR-ed into fp16 1024.0
 // give 1024 + q * 16^j exactly; one FMA recovers q exactly and a second computes
-// q * s + (-z * s), rounded once to fp16. c2 = fp16x2(-z * s) of the group.
-__device__ __forceinline__ void decode_word_b4(uint32_t v, uint32_t s2, uint32_t c2, uint32_t* out) {
+// q * s + (-z * s), rounded once to fp16. c2 = fp16x2(-z * s) of the group. Word w of the half
+// (block w / 4, word q = w % 4 of it): pair c goes to out[16 * (w / 4) + 4c + q].
+__device__ __forceinline__ void decode_word_b4(uint32_t v, uint32_t s2, uint32_t c2, uint32_t* out, int w) {
     constexpr uint32_t kMagic = 0x64006400u;
     constexpr uint32_t kMul[2] = {0x3C003C00u, 0x2C002C00u};   // 1, 1/16
     constexpr uint32_t kAdd[2] = {0xE400E400u, 0xD400D400u};   // -1024, -64
@@ -186,7 +191,7 @@ __device__ __forceinline__ void decode_word_b4(uint32_t v, uint32_t s2, uint32_t
         const int j = c & 1;
         const uint32_t e = and_or(v >> shift, 0x000F000Fu << (4 * j), kMagic);
         const uint32_t q = f16x2_fma(e, kMul[j], kAdd[j]);
-        out[c] = f16x2_fma(q, s2, c2);
+        out[16 * (w >> 2) + 4 * c + (w & 3)] = f16x2_fma(q, s2, c2);
     }
 }
 
@@ -466,10 +471,10 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT>::kThreads, Cfg<BITS, GS, BT>
                         decode_half_b1(words[hh][0], words[hh][1], s2[hh], out);
                     } else if (BITS == 2) {
 #pragma unroll
-                        for (int w = 0; w < 4; ++w) decode_word_b2(words[hh][w], s2[hh], out + 8 * w);
+                        for (int w = 0; w < 4; ++w) decode_word_b2(words[hh][w], s2[hh], out, w);
                     } else {
 #pragma unroll
-                        for (int w = 0; w < 8; ++w) decode_word_b4(words[hh][w], s2[hh], c2[hh], out + 4 * w);
+                        for (int w = 0; w < 8; ++w) decode_word_b4(words[hh][w], s2[hh], c2[hh], out, w);
                     }
                     tmem_st32(lane_base + C::kACol0 + a * 64 + h * 32, out);
                 }

@@ -9,9 +9,9 @@
 // mma.sync sustains ~1000 MACs per clock per SM (one per ~8 clocks per SM sub-partition, also
 // with the decode instructions interleaved) and takes its B operand from registers, so decoded
 // weights need no staging. Its latency is long (~90 clocks when chains restart), so each warp
-// keeps up to eight independent accumulator chains (weight-row octets) in flight; the number
-// of octets per CTA is a template parameter so that a step's chains form one straight-line
-// block the compiler can interleave.
+// keeps several independent accumulator chains (weight-row octets) in flight and each SM
+// sub-partition runs four warps; the number of octets per CTA is a template parameter so that a
+// step's chains form one straight-line block the compiler can interleave.
 //
 // Arithmetic. X is used as stored (bf16); codes are decoded WITHOUT their scale into exact bf16
 // values and the group scale is applied to fp32 group sums afterwards:
@@ -31,12 +31,14 @@
 //     the scales (and zeros) of the step's groups. There is no producer warp: thread 0 issues
 //     the first ring's worth, and afterwards the last warp to finish with a slot refills it
 //     (a shared-memory arrival counter), so no warp ever blocks on a slot being released;
-//   * each of the eight warps takes 64 of the step's 512 K (one group or half of one): it turns
-//     its group's fp16 scales / zeros into fp32 pairs (s, s * c), loads its four X fragments
-//     once with ldmatrix, forms Sx with four MMAs against ones, and runs the decode + MMA
-//     chains of all the tile's octets, their codes loaded ahead of each sub-batch;
-//   * at the end of a tile the eight warps' partial sums are added in a fixed order through
-//     shared memory, then across the cluster, so results do not depend on timing.
+//   * sixteen warps (128 registers each, four per sub-partition to hide latency): warps w and
+//     w + 8 take the same 64 of the step's 512 K (one group or half of one), each for one half
+//     of the tile's octets. A warp turns its group's fp16 scales / zeros for its rows into fp32
+//     pairs (s, s * c), loads its four X fragments once with ldmatrix, forms Sx with four MMAs
+//     against ones, and runs the decode + MMA chains of its octets, their codes loaded ahead of
+//     each sub-batch;
+//   * at the end of a tile the eight K-chunk partial sums of every octet are added in a fixed
+//     order through shared memory, then across the cluster, so results do not depend on timing.
 #pragma once
 
 #include <cuda.h>
@@ -52,13 +54,18 @@
 namespace lowbit {
 namespace smallm {
 
-constexpr int kWarps = 8;                         // each takes 64 K of every step
+constexpr int kKWarps = 8;                        // 64-wide K chunks per step
+// Octet halves per K chunk: with 2, warps w and w + 8 take the same K chunk, each for half the
+// octets (16 warps of 128 registers). Measured on B200 with block-ordered codes, 1 (8 warps)
+// is as fast or faster on the 16-token text-encoder shapes, so it is the one built.
+constexpr int kHalves = 1;
+constexpr int kWarps = kKWarps * kHalves;
 constexpr int kThreads = kWarps * 32;
 constexpr int kStepK = 512;                       // K per ring step
 constexpr int kTokens = 16;
 constexpr int kMaxRows = 128;
 constexpr int kMaxOct = kMaxRows / 8;
-constexpr int kMaxChains = 12;                    // octet chains interleaved per sub-batch
+constexpr int kMaxChains = kHalves == 1 ? 12 : 5;  // octet chains interleaved per sub-batch
 constexpr int kMaxStages = 8;
 constexpr int kXBytes = kTokens * kStepK * 2;     // X slice of one step: 16 KB
 constexpr int kSmemLimit = 227 * 1024;
@@ -100,7 +107,7 @@ bool layout(int rows, int ksplit, Params* p, int* smem_bytes) {
     const uint32_t end = p->z_off + (BITS == 4 ? s_bytes : 0);
     p->stage_bytes = (end + 1023) / 1024 * 1024;
     p->tx_bytes = kXBytes + w_bytes + s_raw * (BITS == 4 ? 2 : 1);
-    const uint32_t scr = kWarps * (rows / 2) * 16;   // per warp: (s, s * c) pairs of its group
+    const uint32_t scr = kWarps * 4 * ((noct + kHalves - 1) / kHalves) * 16;   // per warp: (s, s * c) pairs of its rows
     const uint32_t red = 4 * noct * 512;
     // receive buffer of the octets this rank finishes: [ksplit][ceil(noct / ksplit)][32 lanes]
     const uint32_t part = ksplit > 1 ? ksplit * ((noct + ksplit - 1) / ksplit) * 512 : 0;
@@ -141,7 +148,7 @@ __device__ __forceinline__ void mma_bf16_z(float (&d)[4], const uint32_t (&a)[4]
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.f));
 }
 
-__device__ __forceinline__ void cta_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+__device__ __forceinline__ void cta_bar() { asm volatile("bar.sync 1, %0;" ::"n"(kThreads) : "memory"); }
 
 // Shared-memory counter increment with acquire-release ordering at CTA scope; returns the old value.
 __device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t* p, uint32_t v) {
@@ -157,7 +164,8 @@ __device__ __forceinline__ void st_shared_cluster_v4(uint32_t addr, float4 v) {
                  : "memory");
 }
 
-// Exact bf16 pairs of two neighbouring codes (k, k + 1) at pair index c of a packed word.
+// Exact bf16 pairs of two neighbouring codes (k, k + 1) at pair index c of a packed word (c a
+// compile-time constant after unrolling, so pair 0 needs no shift).
 __device__ __forceinline__ uint32_t dec_u4(uint32_t v, int c) {       // 128 + q
     return and_or(v >> (4 * c), 0x000F000Fu, 0x43004300u);
 }
@@ -176,9 +184,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     using F = Fmt<BITS, GS>;
     constexpr int R = 8 * NOCT;                       // weight rows per tile
     constexpr int HALF = R / 2;                       // (s, s * c) pairs per group
-    constexpr int NB = (NOCT + kMaxChains - 1) / kMaxChains;
-    constexpr int B = (NOCT + NB - 1) / NB;           // octets per sub-batch
-    constexpr int WPS = BITS == 4 ? 8 : BITS == 2 ? 4 : 2;   // code words per lane per octet per step
+    constexpr int NH = (NOCT + kHalves - 1) / kHalves; // octets per warp (its half of the tile)
+    constexpr int HP = 4 * NH;                        // (s, s * c) pairs of a half's rows
+    constexpr int NB = (NH + kMaxChains - 1) / kMaxChains;
+    constexpr int B = (NH + NB - 1) / NB;             // octets per sub-batch
+    constexpr int WPS = BITS == 4 ? 2 : BITS == 2 ? 1 : 2;   // code words per lane per octet per step
     if (threadIdx.x == 0) {
         tma_prefetch_desc(&map_x);
         tma_prefetch_desc(&map_w);
@@ -254,7 +264,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
 
-    const int w = warp;
+    const int w = warp & (kKWarps - 1);      // this warp's 64-wide K chunk of every step
+    const int ob0 = (warp / kKWarps) * NH;   // first octet of this warp's half of the tile
+    const int nh = (NOCT % kHalves == 0) ? NH : min(NH, NOCT - ob0);   // octets it owns
     const int g = lane >> 2;                 // B column (weight row in the octet) / C row
     const int q = lane & 3;
     const int gi = (w * 64) / GS;            // this warp's group within a step
@@ -262,40 +274,44 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t xoff = static_cast<uint32_t>(w * 2048 + tok * 128);
     const int xhalf = lane >> 4;
     // This lane's code bytes in row g of octet 0 of a step (swizzled as the TMA wrote them; the
-    // swizzle depends on the row only through g, so octet o is at a fixed offset from it).
-    uint32_t wb0, wb1;                       // two 16-byte pieces (uint4) or one piece (others)
+    // swizzle depends on the row only through g, so octet o is at a fixed offset from it). 2- and
+    // 4-bit codes are in block order: each 16-byte unit of a row is one block of four words, and
+    // word q of a block is exactly lane q's codes for the block's columns, so a lane loads one
+    // word per block: two blocks (uint4) or one (ternary) per 64-wide K chunk.
+    uint32_t wb0, wb1;                       // the lane's word in each block (binary: 8 bytes)
     constexpr uint32_t kOctStride = BITS == 1 ? 512u : 1024u;
     if (BITS == 4) {
         const int c0 = 2 * (w & 3);
-        wb0 = static_cast<uint32_t>((w >> 2) * R * 128 + g * 128 + ((c0 ^ g) << 4));
-        wb1 = static_cast<uint32_t>((w >> 2) * R * 128 + g * 128 + (((c0 + 1) ^ g) << 4));
+        wb0 = static_cast<uint32_t>((w >> 2) * R * 128 + g * 128 + ((c0 ^ g) << 4) + 4 * q);
+        wb1 = static_cast<uint32_t>((w >> 2) * R * 128 + g * 128 + (((c0 + 1) ^ g) << 4) + 4 * q);
     } else if (BITS == 2) {
-        wb0 = wb1 = static_cast<uint32_t>(g * 128 + ((w ^ g) << 4));
+        wb0 = wb1 = static_cast<uint32_t>(g * 128 + ((w ^ g) << 4) + 4 * q);
     } else {
         wb0 = wb1 = static_cast<uint32_t>(g * 64 + (((w >> 1) ^ ((g >> 1) & 3)) << 4) + (w & 1) * 8);
     }
-    float4* scr = reinterpret_cast<float4*>(smem + p.scr_off) + w * HALF;
+    float4* scr = reinterpret_cast<float4*>(smem + p.scr_off) + warp * HP;
 
-    float acc[NOCT][4];
+    float acc[NH][4];
 #pragma unroll
-    for (int o = 0; o < NOCT; ++o) acc[o][0] = acc[o][1] = acc[o][2] = acc[o][3] = 0.f;
+    for (int o = 0; o < NH; ++o) acc[o][0] = acc[o][1] = acc[o][2] = acc[o][3] = 0.f;
     int it = 0, ti = 0;
+    int s = 0;                               // ring slot of step it, and its fill parity
+    uint32_t ph = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < p.n_tiles; t += gridDim.x, ++ti) {
         for (int c = 0; c < nst; ++c, ++it) {
-            const int s = it % S;
-            ok = ok && __all_sync(0xffffffffu, mbar_wait(&full[s], (it / S) & 1u, abort_flag, p.status));
+            ok = ok && __all_sync(0xffffffffu, mbar_wait(&full[s], ph, abort_flag, p.status));
             if (ok) {
                 const uint8_t* st = ring + s * p.stage_bytes;
                 const uint32_t st_u = smem_u32(st);
-                // this warp's group: fp32 (s, s * c) for every pair of rows of the tile
+                // this warp's group: fp32 (s, s * c) for every pair of rows of its octets
                 {
-                    const __half2* sp = reinterpret_cast<const __half2*>(st + p.s_off) + gi * HALF;
-                    const __half2* zp = reinterpret_cast<const __half2*>(st + p.z_off) + gi * HALF;
+                    const __half2* sp = reinterpret_cast<const __half2*>(st + p.s_off) + gi * HALF + 4 * ob0;
+                    const __half2* zp = reinterpret_cast<const __half2*>(st + p.z_off) + gi * HALF + 4 * ob0;
 #pragma unroll
-                    for (int i0 = 0; i0 < HALF; i0 += 32) {
+                    for (int i0 = 0; i0 < HP; i0 += 32) {
                         const int i = i0 + lane;
-                        if (i < HALF) {
+                        if (i < 4 * nh) {
                             const float2 sf = __half22float2(sp[i]);
                             float c0 = 0.f, c1 = 0.f;
                             if (BITS == 4) {
@@ -326,21 +342,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 const uint8_t* wst = st + p.w_off;
 #pragma unroll
-                for (int ob = 0; ob < NOCT; ob += B) {
+                for (int ob = 0; ob < NH; ob += B) {
                     // codes of the sub-batch's octets for this warp's 64 K
                     uint32_t wd[B][WPS];
 #pragma unroll
                     for (int u = 0; u < B; ++u) {
-                        if (ob + u < NOCT) {
-                            const uint8_t* rp = wst + (ob + u) * kOctStride;
+                        if (ob + u < nh) {
+                            const uint8_t* rp = wst + (ob0 + ob + u) * kOctStride;
                             if (BITS == 4) {
-                                const uint4 v0 = *reinterpret_cast<const uint4*>(rp + wb0);
-                                const uint4 v1 = *reinterpret_cast<const uint4*>(rp + wb1);
-                                wd[u][0] = v0.x; wd[u][1] = v0.y; wd[u][2] = v0.z; wd[u][3] = v0.w;
-                                wd[u][4] = v1.x; wd[u][5] = v1.y; wd[u][6] = v1.z; wd[u][7] = v1.w;
+                                wd[u][0] = *reinterpret_cast<const uint32_t*>(rp + wb0);
+                                wd[u][1] = *reinterpret_cast<const uint32_t*>(rp + wb1);
                             } else if (BITS == 2) {
-                                const uint4 v = *reinterpret_cast<const uint4*>(rp + wb0);
-                                wd[u][0] = v.x; wd[u][1] = v.y; wd[u][2] = v.z; wd[u][3] = v.w;
+                                wd[u][0] = *reinterpret_cast<const uint32_t*>(rp + wb0);
                             } else {
                                 const uint2 v = *reinterpret_cast<const uint2*>(rp + wb0);
                                 wd[u][0] = v.x; wd[u][1] = v.y;
@@ -352,14 +365,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int j = 0; j < 4; ++j) {
 #pragma unroll
                         for (int u = 0; u < B; ++u) {
-                            if (ob + u < NOCT) {
+                            if (ob + u < nh) {
                                 uint32_t b0, b1;
-                                if (BITS == 4) {
-                                    b0 = dec_u4(wd[u][2 * j], q);
-                                    b1 = dec_u4(wd[u][2 * j + 1], q);
-                                } else if (BITS == 2) {
-                                    b0 = dec_t2(wd[u][j], q);
-                                    b1 = dec_t2(wd[u][j], q + 4);
+                                if (BITS == 4) {           // block j / 2, pairs 2(j % 2) and + 1
+                                    b0 = dec_u4(wd[u][j >> 1], 2 * (j & 1));
+                                    b1 = dec_u4(wd[u][j >> 1], 2 * (j & 1) + 1);
+                                } else if (BITS == 2) {    // the chunk's block, pairs 2j and 2j + 1
+                                    b0 = dec_t2(wd[u][0], 2 * j);
+                                    b1 = dec_t2(wd[u][0], 2 * j + 1);
                                 } else {
                                     const int pc = (j & 1) * 8 + q;
                                     b0 = dec_b1(wd[u][j >> 1], pc);
@@ -373,7 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (ob == 0) __syncwarp();   // the scale pairs above are written
 #pragma unroll
                     for (int u = 0; u < B; ++u) {
-                        if (ob + u < NOCT) {
+                        if (ob + u < nh) {
                             const float4 sc = scr[4 * (ob + u) + q];
                             float* d = acc[ob + u];
                             d[0] = fmaf(sc.x, T[u][0], d[0]);
@@ -391,54 +404,63 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             __syncwarp();
-            // Release the slot; the last warp out queues ring step it + look (into the slot of step
-            // it + look - S <= it, which every warp has left).
-            if (lane == 0) {
+            // Release the slot; the last warp out queues ring step it + look = it + S into it. Once
+            // no step is left to queue, this slot (and every later step's) needs no count.
+            if (lane == 0 && it + look < total) {
                 const uint32_t prev = atom_add_acq_rel(&cnt[s], 1);
-                if ((prev & (kWarps - 1)) == kWarps - 1 && it + look < total && !*abort_flag) {
+                if ((prev & (kWarps - 1)) == kWarps - 1 && !*abort_flag) {
                     issue(it + look, true, true);
-                    iss[(it + look) % S] += 1;
+                    iss[s] += 1;
                 }
+            }
+            if (++s == S) {
+                s = 0;
+                ph ^= 1u;
             }
         }
 
-        // ---- tile end: sum the eight warps' partials in a fixed order. On a CTA's only tile the
-        // drained ring holds all eight: one exchange, ((((w0 + w1) + w2) + ...) + w7). Otherwise
-        // the ring already holds the next tile's steps and `red` takes two rounds:
-        // (w + (w + 4)) for w < 4, then ((0 + 1) + 2) + 3.
+        // ---- tile end: every octet's eight K-chunk partials (one per warp of its half) are added
+        // in a fixed order. On a CTA's only tile the drained ring holds all eight: one exchange,
+        // ((((c0 + c1) + c2) + ...) + c7). Otherwise the ring already holds the next tile's steps
+        // and `red` takes two rounds: (c + (c + 4)) for chunks c < 4, then ((0 + 1) + 2) + 3.
         grid_dependency_wait();   // Y may still be read by the kernel this one overlaps
-        const bool one_round = my_tiles == 1 && static_cast<uint32_t>(S) * p.stage_bytes >= kWarps * NOCT * 512u;
+        const bool one_round =
+            my_tiles == 1 && static_cast<uint32_t>(S) * p.stage_bytes >= kKWarps * NOCT * 512u;
         float4* rbuf = one_round ? reinterpret_cast<float4*>(ring) : red;
-        const int nslot = one_round ? kWarps : 4;
+        const int nslot = one_round ? kKWarps : 4;
         cta_bar();                // the ring is drained / the previous tile's readers of `red` are done
         if (one_round || w >= 4) {
             const int slot = one_round ? w : w - 4;
 #pragma unroll
-            for (int o = 0; o < NOCT; ++o)
-                rbuf[(slot * NOCT + o) * 32 + lane] = make_float4(acc[o][0], acc[o][1], acc[o][2], acc[o][3]);
+            for (int o = 0; o < NH; ++o)
+                if (o < nh)
+                    rbuf[(slot * NOCT + ob0 + o) * 32 + lane] = make_float4(acc[o][0], acc[o][1], acc[o][2], acc[o][3]);
         }
         cta_bar();
         if (!one_round) {
             if (w < 4) {
 #pragma unroll
-                for (int o = 0; o < NOCT; ++o) {
-                    const float4 v = red[(w * NOCT + o) * 32 + lane];
-                    acc[o][0] += v.x;
-                    acc[o][1] += v.y;
-                    acc[o][2] += v.z;
-                    acc[o][3] += v.w;
+                for (int o = 0; o < NH; ++o) {
+                    if (o < nh) {
+                        const float4 v = red[(w * NOCT + ob0 + o) * 32 + lane];
+                        acc[o][0] += v.x;
+                        acc[o][1] += v.y;
+                        acc[o][2] += v.z;
+                        acc[o][3] += v.w;
+                    }
                 }
             }
             cta_bar();
             if (w < 4) {
 #pragma unroll
-                for (int o = 0; o < NOCT; ++o)
-                    red[(w * NOCT + o) * 32 + lane] = make_float4(acc[o][0], acc[o][1], acc[o][2], acc[o][3]);
+                for (int o = 0; o < NH; ++o)
+                    if (o < nh)
+                        red[(w * NOCT + ob0 + o) * 32 + lane] = make_float4(acc[o][0], acc[o][1], acc[o][2], acc[o][3]);
             }
             cta_bar();
         }
 #pragma unroll
-        for (int o = 0; o < NOCT; ++o) acc[o][0] = acc[o][1] = acc[o][2] = acc[o][3] = 0.f;
+        for (int o = 0; o < NH; ++o) acc[o][0] = acc[o][1] = acc[o][2] = acc[o][3] = 0.f;
 
         const int n0 = t * R;
         auto store = [&](int o, float4 v) {
@@ -455,7 +477,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         auto tile_sum = [&](int o) {
             float4 v = rbuf[o * 32 + lane];
 #pragma unroll
-            for (int r = 1; r < kWarps; ++r) {
+            for (int r = 1; r < kKWarps; ++r) {
                 if (r >= nslot) break;
                 const float4 u = rbuf[(r * NOCT + o) * 32 + lane];
                 v.x += u.x;
@@ -466,19 +488,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             return v;
         };
         if (ks == 1) {
-            for (int o = w; o < NOCT; o += kWarps) store(o, tile_sum(o));
+            for (int o = warp; o < NOCT; o += kWarps) store(o, tile_sum(o));
         } else {
             // Octet o is finished by rank o % ks: every rank stores its tile sum of o straight into
             // that rank's receive buffer (slot [own rank][o / ks]); after a cluster barrier the
             // finishing rank adds the slots in rank order; a second barrier keeps the buffers
             // (and every CTA) alive until all ranks have read them.
             const int per = (NOCT + ks - 1) / ks;
-            for (int o = w; o < NOCT; o += kWarps) {
+            for (int o = warp; o < NOCT; o += kWarps) {
                 const uint32_t slot = smem_u32(part + ((rank * per + o / ks) * 32 + lane));
                 st_shared_cluster_v4(map_shared_rank(slot, o % ks), tile_sum(o));
             }
             cluster_sync_all();
-            for (int o = w; o < NOCT; o += kWarps) {
+            for (int o = warp; o < NOCT; o += kWarps) {
                 if (o % ks != rank) continue;
                 const int li = o / ks;
                 float4 sum = part[li * 32 + lane];

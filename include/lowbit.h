@@ -17,14 +17,22 @@
  *
  * Packed code layout (uint32 words, packed along K; produced by lowbit_pack):
  *   cpw = 32 / bits codes per word; row n of W owns words [n*K/cpw, (n+1)*K/cpw).
- *   The code of column k is in word k / cpw at offset i = k % cpw, in bits
- *   [pos, pos + bits) with pos = (i % 2) * 16 + (i / 2) * bits: even offsets fill the low
- *   16 bits and odd offsets the high 16 bits, each half LSB-first. Stored fields:
- *   binary +1 -> 1, -1 -> 0; ternary t -> t + 1 (3 is invalid); uint4 q -> q.
+ *   Offset i of a word (0 .. cpw-1) occupies bits [pos, pos + bits) with
+ *   pos = (i % 2) * 16 + (i / 2) * bits: offsets 2p and 2p + 1 ("pair p") fill the low and
+ *   the high 16 bits, each half LSB-first. Which column an offset holds:
+ *   - block order (2- and 4-bit rows, words taken in blocks of four, a block spanning
+ *     4 * cpw columns: 32 for uint4, 64 for ternary): in word q (0..3) of block b, pair p
+ *     holds columns 4*cpw*b + 8p + 2q (low half) and 4*cpw*b + 8p + 2q + 1 (high half);
+ *   - plain order (every binary word, and the words after the last whole block of a 2- or
+ *     4-bit row, i.e. when K is not a multiple of 4 * cpw): word j, offset i holds column
+ *     cpw * j + i.
+ *   Stored fields: binary +1 -> 1, -1 -> 0; ternary t -> t + 1 (3 is invalid); uint4 q -> q.
  *   (The pages pack codes along K into uint32 words -- Bonsai-Image-Demo PR #20, GemLite
- *   int2 layout note; image-studio backend.md, checkpoint layout -- but leave the bit order
- *   open. This order puts the two codes of a K pair in the two bf16 halves of one 32-bit
- *   register, so a decoder builds bf16x2 operands with one mask per pair.)
+ *   int2 layout note; image-studio backend.md, checkpoint layout -- but leave the order
+ *   inside the words open. Pairs put two K-neighbours in the two 16-bit halves of one
+ *   register, so one mask builds a bf16x2 / fp16x2 operand; block order makes word q of a
+ *   block exactly the codes lane q of a warp-level m16n8k16 MMA needs from that block, so
+ *   the small-M kernel loads one 32-bit word per lane per block.)
  *
  * Scale / zero layout: fp16, group-major [K/group_size][N]: s(n, k) = scales[(k/g)*N + n].
  * X: bf16 row-major [M][K]. Y: bf16 row-major [M][N].
