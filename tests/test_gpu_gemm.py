@@ -226,6 +226,27 @@ def test_full_size_sampled(spec):
     print(f"\n{spec.name} M={spec.M} K={spec.K} N={spec.N}: max err/bound {worst:.3f}")
 
 
+@pytest.mark.parametrize("bits,gs", [(4, 64), (2, 128), (1, 128)])
+def test_second_wave_tiles(bits, gs):
+    """512 x 2048 -> 9728: 2 x 76 = 152 tiles of 256 tokens x 128 rows. On a 148-SM B200 the
+    persistent grid gives the last 4 tiles (tokens 256.., rows 9216..) to CTAs that already
+    finished one, after their accumulator is drained; every output of those tiles is checked,
+    plus random outputs elsewhere."""
+    spec = spec_for(bits, gs, 512, 2048, 9728, seed=7)
+    prob = synth.make_problem(spec)
+    x, packed, s, z = _gpu.dev_problem(prob)
+    y = _gpu.y_to_f64(lb.gemm(x, packed, s, z, bits, gs))
+    assert lb.device_status() == 0
+    tm, tn = np.meshgrid(np.arange(256, 512), np.arange(9216, 9728), indexing="ij")
+    r = np.random.default_rng(3)
+    ms = np.concatenate([tm.ravel(), r.integers(0, 512, 8192)])
+    ns = np.concatenate([tn.ravel(), r.integers(0, 9728, 8192)])
+    ref = oracle.gemm_entries(prob.x_bf16, _gpu.oracle_packed(prob), prob.scales, prob.zeros, spec.N, bits, gs,
+                              ms, ns)
+    rms = float(np.sqrt(np.mean(ref * ref)))
+    _gpu.check_close(y[ms, ns], ref, rms=rms, what=f"second-wave tiles bits={bits}")
+
+
 def chain_distinct():
     seen = {}
     for s in synth.chain_linears():
