@@ -9,9 +9,9 @@
 // mma.sync sustains ~1000 MACs per clock per SM (one per ~8 clocks per SM sub-partition, also
 // with the decode instructions interleaved) and takes its B operand from registers, so decoded
 // weights need no staging. Its latency is long (~90 clocks when chains restart), so each warp
-// keeps several independent accumulator chains (weight-row octets) in flight and each SM
-// sub-partition runs four warps; the number of octets per CTA is a template parameter so that a
-// step's chains form one straight-line block the compiler can interleave.
+// keeps several independent accumulator chains (weight-row octets) in flight; the number of
+// octets per CTA is a template parameter so that a step's chains form one straight-line block
+// the compiler can interleave.
 //
 // Arithmetic. X is used as stored (bf16); codes are decoded WITHOUT their scale into exact bf16
 // values and the group scale is applied to fp32 group sums afterwards:
@@ -31,12 +31,12 @@
 //     the scales (and zeros) of the step's groups. There is no producer warp: thread 0 issues
 //     the first ring's worth, and afterwards the last warp to finish with a slot refills it
 //     (a shared-memory arrival counter), so no warp ever blocks on a slot being released;
-//   * sixteen warps (128 registers each, four per sub-partition to hide latency): warps w and
-//     w + 8 take the same 64 of the step's 512 K (one group or half of one), each for one half
-//     of the tile's octets. A warp turns its group's fp16 scales / zeros for its rows into fp32
-//     pairs (s, s * c), loads its four X fragments once with ldmatrix, forms Sx with four MMAs
-//     against ones, and runs the decode + MMA chains of its octets, their codes loaded ahead of
-//     each sub-batch;
+//   * eight warps, each taking 64 of the step's 512 K (one group or half of one) for all the
+//     tile's octets (kHalves = 2 instead runs sixteen warps of 128 registers, warps w and w + 8
+//     sharing a K chunk with half the octets each). A warp turns its group's fp16 scales /
+//     zeros for its rows into fp32 pairs (s, s * c), loads its four X fragments once with
+//     ldmatrix, forms Sx with four MMAs against ones, and runs the decode + MMA chains of its
+//     octets, each lane loading one 32-bit code word per block of block-ordered codes;
 //   * at the end of a tile the eight K-chunk partial sums of every octet are added in a fixed
 //     order through shared memory, then across the cluster, so results do not depend on timing.
 #pragma once
@@ -294,11 +294,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     float acc[NH][4];
 #pragma unroll
     for (int o = 0; o < NH; ++o) acc[o][0] = acc[o][1] = acc[o][2] = acc[o][3] = 0.f;
-    int it = 0, ti = 0;
+    int it = 0;
     int s = 0;                               // ring slot of step it, and its fill parity
     uint32_t ph = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < p.n_tiles; t += gridDim.x, ++ti) {
+    for (int t = blockIdx.x; t < p.n_tiles; t += gridDim.x) {
         for (int c = 0; c < nst; ++c, ++it) {
             ok = ok && __all_sync(0xffffffffu, mbar_wait(&full[s], ph, abort_flag, p.status));
             if (ok) {

@@ -97,8 +97,13 @@ lowbit_status lowbit_unpack(const uint32_t* packed, int64_t N, int64_t K, int bi
  * (M*K*2 bytes, rounded up to 256) plus one float per row (rounded up to 256). 0 if M or K < 0. */
 size_t lowbit_gemm_workspace_size(int64_t M, int64_t K);
 
-/* Y = X * W^T on `stream` (asynchronous; never synchronises). Two kernels run in order on the
- * stream: the X -> fp16 conversion into `workspace`, then the GEMM.
+/* Y = X * W^T on `stream` (asynchronous; never synchronises). For M > 16 two kernels run in
+ * order on the stream: the X -> fp16 conversion into `workspace`, then the GEMM; for M <= 16 one
+ * kernel reads X directly. Kernels are programmatic dependents of the work enqueued before
+ * them: for M <= 16 the GEMM starts streaming Wp, scales and zeros before that work has
+ * finished (X is read only after it), so Wp, scales and zeros must not be written by the
+ * kernel enqueued immediately before the call (lowbit_pack returns only after its kernel has
+ * completed, so packing right before is fine).
  *   X          [M][K]            bf16, device, 16-byte aligned
  *   Wp         [N][K*bits/32]    uint32 packed codes, device, 16-byte aligned
  *   scales     [K/group_size][N] fp16, device, 16-byte aligned
