@@ -23,6 +23,19 @@ def test_pack_unpack_bit_exact(bits, N, K):
     assert np.array_equal(back.cpu().numpy(), codes)
 
 
+@pytest.mark.parametrize("bits,K", [(4, 40), (4, 104), (2, 80), (2, 112), (2, 48)])
+def test_pack_rows_with_plain_tail_words(bits, K):
+    """Rows whose word count is not a multiple of four: whole blocks in block order, then the
+    remaining words in plain order."""
+    N = 11
+    codes = _pins.random_codes(N, K, bits, seed=K + 7 * bits)
+    want, bad = oracle.pack(codes, bits)
+    assert bad == 0
+    got = lb.pack(torch.from_numpy(codes).cuda(), bits)
+    assert np.array_equal(got.cpu().numpy().view(np.uint32), want)
+    assert np.array_equal(lb.unpack(got, N, K, bits).cpu().numpy(), codes)
+
+
 def test_pack_golden_words():
     for bits, K, N, codes, words in _pins.load_golden_pack():
         got = lb.pack(torch.from_numpy(codes).cuda(), bits).cpu().numpy().view(np.uint32)
