@@ -496,13 +496,22 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT>::kThreads, Cfg<BITS, GS, BT>
         grid_dependency_wait();                      // before the first global access
         constexpr int kChunk = (C::kEpiCols >= 32) ? 32 : 16;
         uint32_t tcount = 0;
+        constexpr int kChunks = C::kEpiCols / kChunk;
         for (int t = 0; t < my_tiles; ++t, ++tcount) {
             const int tile = static_cast<int>(blockIdx.x) + t * tile_step;
             const uint32_t b = tcount % NACC, acc_ph = (tcount / NACC) & 1u;
-            if (!__all_sync(0xffffffffu, mbar_wait(&accfull[b], acc_ph, abort_flag, status))) break;
-            tc_fence_after();
             const int m0 = (tile / p.n_tiles) * BT + col0;   // first token of this thread's columns
             const int n = (tile % p.n_tiles) * p.rows + row;
+            // Lane j of the warp holds the row factor of token m0 + c0 + j of every chunk c0,
+            // requested before waiting for the accumulator so the loads overlap the MMAs.
+            float mul[kChunks];
+#pragma unroll
+            for (int ci = 0; ci < kChunks; ++ci) {
+                const int mj = m0 + ci * kChunk + lane;
+                mul[ci] = (!split && lane < kChunk && mj < p.M) ? p.rowmul[mj] : 1.0f;
+            }
+            if (!__all_sync(0xffffffffu, mbar_wait(&accfull[b], acc_ph, abort_flag, status))) break;
+            tc_fence_after();
             if (!split) {
                 // Read the whole slice into registers (scaled, rounded to bf16), hand the
                 // accumulator back to the MMA issuer, then store: the stores of this tile
@@ -516,8 +525,7 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT>::kThreads, Cfg<BITS, GS, BT>
                     } else {
                         tmem_ld16(lane_base + b * BT + col0 + c0, *reinterpret_cast<uint32_t(*)[16]>(v));
                     }
-                    const int mj = m0 + c0 + lane;           // lane j fetches token m0 + c0 + j's factor
-                    const float mul_j = (lane < kChunk && mj < p.M) ? p.rowmul[mj] : 1.0f;
+                    const float mul_j = mul[c0 / kChunk];
                     tmem_wait_ld();
 #pragma unroll
                     for (int j = 0; j < kChunk; j += 2) {
@@ -569,6 +577,12 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT>::kThreads, Cfg<BITS, GS, BT>
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&accempty[b]);
+                // The row factors of the tile's tokens, for the reduction below, go to the weight
+                // ring (every stage has been decoded by now): the reduction then reads them from
+                // shared memory instead of waiting on a global load behind each store.
+                const int te = (warp - C::kFirstEpiWarp) * 32 + lane;
+                const int mt = (tile / p.n_tiles) * BT;
+                if (te < BT) reinterpret_cast<float*>(wring)[te] = (mt + te < p.M) ? p.rowmul[mt + te] : 1.0f;
             }
         }
     }
@@ -591,25 +605,48 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT>::kThreads, Cfg<BITS, GS, BT>
             const int cb = rank * per_rank;
             const int ce = min(BT, cb + per_rank);
             const uint32_t part0 = smem_u32(smem);
+            const float* fac = reinterpret_cast<const float*>(wring);
             if (row < p.rows && n < p.N) {
-                for (int c = cb + 4 * epart; c < ce; c += 4 * C::kEpiParts) {
-                    if (m0 + c >= p.M) break;
-                    const int pc = (c >> 2) ^ (row & C::kPartSwizzle);
-                    const uint32_t off = static_cast<uint32_t>((row * BT + pc * 4) * 4);
-                    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-                    for (int q = 0; q < p.ksplit; ++q) {
-                        const float4 v = ld_shared_cluster_v4(map_shared_rank(part0 + off, q));
-                        acc.x += v.x;
-                        acc.y += v.y;
-                        acc.z += v.z;
-                        acc.w += v.w;
-                    }
-                    const float a4[4] = {acc.x, acc.y, acc.z, acc.w};
+                // kPass 4-column groups per pass (two where registers allow): every rank's
+                // 16-byte chunk of them is requested before any is added, then the ranks are
+                // summed in order and the sums scaled by the row factors staged above and stored.
+                constexpr int kMaxRanks = 8;
+                constexpr int kPass = C::kCtasPerSm == 2 ? 1 : 2;
+                constexpr int kStep = 4 * C::kEpiParts;
+                const int ks = p.ksplit;
+                const int cend = min(ce, p.M - m0);
+                for (int c = cb + 4 * epart; c < cend; c += kPass * kStep) {
+                    float4 v[kPass][kMaxRanks];
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const int m = m0 + c + j;
-                        if (m < p.M)
-                            p.Y[static_cast<size_t>(m) * p.N + n] = __float2bfloat16_rn(a4[j] * p.rowmul[m]);
+                    for (int h = 0; h < kPass; ++h) {
+                        const int cc = c + h * kStep;
+                        const int pc = (cc >> 2) ^ (row & C::kPartSwizzle);
+                        const uint32_t off = static_cast<uint32_t>((row * BT + pc * 4) * 4);
+#pragma unroll
+                        for (int q = 0; q < kMaxRanks; ++q)
+                            if (q < ks && cc < cend) v[h][q] = ld_shared_cluster_v4(map_shared_rank(part0 + off, q));
+                    }
+#pragma unroll
+                    for (int h = 0; h < kPass; ++h) {
+                        const int cc = c + h * kStep;
+                        if (cc >= cend) break;
+                        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                        for (int q = 0; q < kMaxRanks; ++q) {
+                            if (q < ks) {
+                                acc.x += v[h][q].x;
+                                acc.y += v[h][q].y;
+                                acc.z += v[h][q].z;
+                                acc.w += v[h][q].w;
+                            }
+                        }
+                        const float a4[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const int m = m0 + cc + j;
+                            if (m < p.M)
+                                p.Y[static_cast<size_t>(m) * p.N + n] = __float2bfloat16_rn(a4[j] * fac[cc + j]);
+                        }
                     }
                 }
             }
