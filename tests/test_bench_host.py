@@ -94,3 +94,28 @@ def test_reference_arm_other_ranks_exit_quietly():
                    {"RANK": "1", "WORLD_SIZE": "2"})
     assert r.returncode == 0, r.stderr
     assert r.stdout.strip() == ""
+
+
+def _fake_tree(tmp_path, kernel_text, traffic):
+    csrc = tmp_path / "bit_weight_only_w2_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (csrc / "k.cu").write_text(kernel_text)
+    (tmp_path / "include").mkdir()
+    (tmp_path / "include" / "lowbit.h").write_text("/* header */\n")
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(traffic))
+
+
+def test_measured_traffic_follows_the_kernel_sources(tmp_path, monkeypatch):
+    """roofline.traffic is reported only while the CUDA sources hash to the captured ones."""
+    _fake_tree(tmp_path, "__global__ void k() {}\n", {})
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    h = bench.kernel_source_hash()
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(
+        {"w": {"dram_bytes_per_launch": 123.0, "source_sha256": h}}))
+    assert bench.measured_traffic("w") == 123.0
+    assert bench.measured_traffic("other") is None
+    (tmp_path / "bit_weight_only_w2_b200" / "csrc" / "k.cu").write_text("__global__ void k() { }\n")
+    assert bench.kernel_source_hash() != h
+    assert bench.measured_traffic("w") is None          # a changed kernel invalidates the capture
+
