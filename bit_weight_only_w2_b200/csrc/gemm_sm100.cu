@@ -898,15 +898,17 @@ bool make_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, int elem_bytes, co
 int cluster_capacity(const void* kernel, int ks, int threads, int smem_bytes) {
     struct Entry {
         const void* fn;
-        int ks, cap;
+        int dev, ks, cap;
     };
     static Entry cache[64];
     static int used = 0;
     static std::mutex mu;
+    int dev = 0;
+    cudaGetDevice(&dev);
     {
         std::lock_guard<std::mutex> lock(mu);
         for (int i = 0; i < used; ++i)
-            if (cache[i].fn == kernel && cache[i].ks == ks) return cache[i].cap;
+            if (cache[i].fn == kernel && cache[i].dev == dev && cache[i].ks == ks) return cache[i].cap;
     }
     int n = 0;
     cudaLaunchConfig_t cfg = {};
@@ -925,19 +927,25 @@ int cluster_capacity(const void* kernel, int ks, int threads, int smem_bytes) {
         n = num_sms() / ks;
     }
     std::lock_guard<std::mutex> lock(mu);
-    if (used < 64) cache[used++] = Entry{kernel, ks, n};
+    if (used < 64) cache[used++] = Entry{kernel, dev, ks, n};
     return n;
 }
 
+// SM count of the current device (cached per device; 148 if the query fails).
 int num_sms() {
-    static int sms = 0;
-    if (!sms) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        if (sms <= 0) sms = 148;
+    static std::atomic<int> sms[64];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) dev = 0;
+    int n = sms[dev].load(std::memory_order_relaxed);
+    if (n <= 0) {
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+            cudaGetLastError();
+            n = 148;
+        }
+        sms[dev].store(n, std::memory_order_relaxed);
     }
-    return sms;
+    return n;
 }
 
 namespace {

@@ -41,14 +41,19 @@ bool prepare(const void* fn) {
     return true;
 }
 
-// Clusters of `ks` CTAs that fit on the device at once (one CTA per SM), cached per entry point
-// family (all octet counts of a format share the occupancy of one CTA per SM).
+// Clusters of `ks` CTAs that fit on the current device at once (one CTA per SM), cached per
+// device and entry point family (all octet counts of a format share the occupancy of one CTA
+// per SM).
 int cluster_capacity(const void* fn, int bits, int gs, int ks) {
-    static int cache[3][2][9] = {};
+    constexpr int kDevices = 16;
+    static int cache[kDevices][3][2][9] = {};
     const int bi = bits == 1 ? 0 : bits == 2 ? 1 : 2, gi = gs == 64 ? 0 : 1;
-    {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const bool cached = dev >= 0 && dev < kDevices;
+    if (cached) {
         std::lock_guard<std::mutex> lock(g_mu);
-        if (cache[bi][gi][ks] > 0) return cache[bi][gi][ks];
+        if (cache[dev][bi][gi][ks] > 0) return cache[dev][bi][gi][ks];
     }
     int n = 0;
     cudaLaunchConfig_t cfg = {};
@@ -67,8 +72,10 @@ int cluster_capacity(const void* fn, int bits, int gs, int ks) {
         n = num_sms() / ks;
     }
     if (n <= 0) n = 1;
-    std::lock_guard<std::mutex> lock(g_mu);
-    cache[bi][gi][ks] = n;
+    if (cached) {
+        std::lock_guard<std::mutex> lock(g_mu);
+        cache[dev][bi][gi][ks] = n;
+    }
     return n;
 }
 
