@@ -366,14 +366,12 @@ def run_lowbit(args, specs, workload):
     if lb.device_status() != 0:
         raise RuntimeError("kernel timeout reported during the timed steps")
 
-    # Per-launch durations for the roofline. Tensor-bound workloads: each linear timed on the
-    # launching stream with its own events, over two passes (inputs larger than L2). HBM-bound
-    # workloads: the launches run back to back over rotating weight copies, as in the timed
-    # steps, and a launch's duration is the pass time over the number of linears.
-    # Each distinct linear is captured `reps` times back to back in one graph (rotating weight
-    # copies where there are several) and the graph is replayed twice; a launch's duration is
-    # the replay time over `reps`. Each launch is one lowbit_gemm call: for more than 16 tokens
-    # that is the X conversion pass plus the GEMM kernel, for at most 16 the GEMM kernel alone.
+    # Per-launch durations for the roofline: each distinct linear is captured `reps` times back
+    # to back in one graph (rotating weight copies where there are several, so weights stream
+    # from HBM as in the timed steps), the graph is replayed twice on the launching stream, and a
+    # launch's duration is the replay time over `reps`. Each launch is one lowbit_gemm call: for
+    # more than 16 tokens that is the X conversion pass plus the GEMM kernel, for at most 16 the
+    # GEMM kernel alone.
     per = []
     seen = {}
     for it in items:
