@@ -266,7 +266,8 @@ def run_reference(args, specs, workload):
         times.append(dt)
     t = sum(times)
     value = flops * args.steps / t / 1e12
-    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * t / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": workload, "sample_rows_per_shape": rows},
@@ -366,40 +367,71 @@ def run_lowbit(args, specs, workload):
     if lb.device_status() != 0:
         raise RuntimeError("kernel timeout reported during the timed steps")
 
-    # Per-launch durations for the roofline: each distinct linear is captured `reps` times back
-    # to back in one graph (rotating weight copies where there are several, so weights stream
-    # from HBM as in the timed steps), the graph is replayed twice on the launching stream, and a
-    # launch's duration is the replay time over `reps`. Each launch is one lowbit_gemm call: for
-    # more than 16 tokens that is the X conversion pass plus the GEMM kernel, for at most 16 the
-    # GEMM kernel alone.
-    per = []
-    seen = {}
-    for it in items:
-        seen.setdefault((it["spec"].M, it["spec"].K, it["spec"].N), it)
-    for it in seen.values():
-        reps = max(10, copies)
+    # Per-launch durations for the roofline. For each distinct shape, graph A holds `reps`
+    # back-to-back lowbit_gemm calls (rotating weight copies where there are several, so weights
+    # stream from HBM as in the timed steps) and graph B one lowbit_gemm_batch of the same `reps`
+    # linears sharing one X, which the library converts once. A sample replays a graph
+    # `replays` times between two events on the launching stream; the per-launch time is the
+    # median over samples of sample time / (replays * reps). For more than 16 tokens a call is
+    # the X conversion pass plus the GEMM kernel: the conversion's time is (A - B) / (reps - 1)
+    # per launch and the GEMM kernel's is the call's minus that. At most 16 tokens a call is the
+    # small-M GEMM kernel alone.
+    def time_graph(gph, per_sample, samples=9, replays=5, warm=2):
+        for _ in range(warm):
+            gph.replay()
+        torch.cuda.synchronize(device)
+        ts = []
+        for _ in range(samples):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(replays):
+                gph.replay()
+            e1.record(stream)
+            torch.cuda.synchronize(device)
+            ts.append(e0.elapsed_time(e1) / (replays * per_sample))
+        return statistics.median(ts)
+
+    def capture(fn):
         gph = torch.cuda.CUDAGraph()
         cap_stream.wait_stream(stream)
         with torch.cuda.stream(cap_stream):
             with torch.cuda.graph(gph, stream=cap_stream):
-                for i in range(reps):
-                    w_p, w_s, w_z = it["reps"][i % copies]
-                    lb.gemm(it["x"], w_p, w_s, w_z, it["spec"].bits, it["spec"].group_size, out=it["y"])
+                fn()
         stream.wait_stream(cap_stream)
-        gph.replay()
-        torch.cuda.synchronize(device)
-        for _ in range(2):
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            gph.replay()
-            e1.record(stream)
-            torch.cuda.synchronize(device)
-            ms = e0.elapsed_time(e1) / reps
-            per.extend((sp, ms) for sp in [s for s in specs if (s.M, s.K, s.N) == (it["spec"].M, it["spec"].K, it["spec"].N)])
-        del gph
-    launch_ms = sum(ms for _, ms in per) / len(per)
-    launch_flops = sum(sp.flops for sp, _ in per) / len(per)
-    launch_bytes = sum(sp.algorithmic_bytes() for sp, _ in per) / len(per)
+        return gph
+
+    shape_times = {}
+    seen = {}
+    for it in items:
+        seen.setdefault((it["spec"].M, it["spec"].K, it["spec"].N), it)
+    for key, it in seen.items():
+        reps = max(10, copies)
+        sp = it["spec"]
+
+        def calls():
+            for i in range(reps):
+                w_p, w_s, w_z = it["reps"][i % copies]
+                lb.gemm(it["x"], w_p, w_s, w_z, sp.bits, sp.group_size, out=it["y"])
+
+        g_a = capture(calls)
+        t_call = time_graph(g_a, reps)
+        del g_a
+        t_conv = 0.0
+        if sp.M > 16:
+            shared = [lb.make_desc(it["x"], *it["reps"][i % copies], it["y"], sp.bits, sp.group_size)
+                      for i in range(reps)]
+            g_b = capture(lambda: lb.gemm_batch(shared, device))
+            t_shared = time_graph(g_b, reps)
+            del g_b
+            t_conv = max(0.0, (t_call - t_shared) * reps / (reps - 1))
+        shape_times[key] = (t_call, t_call - t_conv, t_conv, reps)
+    per = [(s, *shape_times[(s.M, s.K, s.N)][:3]) for s in specs]     # (spec, call, gemm, conversion) ms
+    launch_ms = sum(c for _, c, _, _ in per) / len(per)
+    gemm_ms = sum(g for _, _, g, _ in per) / len(per)
+    conv_ms = sum(v for _, _, _, v in per) / len(per)
+    launch_flops = sum(sp.flops for sp, _, _, _ in per) / len(per)
+    launch_bytes = sum(sp.algorithmic_bytes() for sp, _, _, _ in per) / len(per)
+    launches_timed = sum(2 * 9 * 5 * r if k[0] > 16 else 9 * 5 * r for k, (_, _, _, r) in shape_times.items())
 
     # End to end through the public API, as a user would pipeline it: each step copies every
     # linear's activations in (pinned host -> device, copy stream), runs lowbit_gemm per linear
@@ -472,29 +504,37 @@ def run_lowbit(args, specs, workload):
                "mode": ("copies on two streams overlapping lowbit_gemm per linear" if pipelined
                         else "copy in, one lowbit_gemm_batch, copy out")}
 
-    long_step = ms_step >= 5.0
     traffic = measured_traffic(workload)
+    burst = peaks.get("bf16_tflops")
     if hbm_bound:
         peak_bw = peaks.get("hbm_gbs")
         achieved = launch_bytes / (launch_ms * 1e-3) / 1e9
         roofline = {"bound": "hbm", "achieved": achieved, "peak": peak_bw, "unit": "GB/s",
                     "frac": achieved / peak_bw, "traffic": traffic,
                     "peak_source": f"{peak_src} HBM copy bandwidth", "kernel": "lowbit_smallm_kernel",
-                    "launches_timed": len(per), "algorithmic_mb_per_launch": launch_bytes / 1e6,
+                    "us_per_launch": launch_ms * 1e3, "launches_timed": launches_timed,
+                    "algorithmic_mb_per_launch": launch_bytes / 1e6,
                     "algorithmic_gflop_per_launch": launch_flops / 1e9,
                     "tflops_per_launch": launch_flops / (launch_ms * 1e-3) / 1e12,
                     "weight_copies_rotated": copies}
     else:
-        peak_tf = peaks.get("bf16_tflops_sustained" if long_step else "bf16_tflops")
-        achieved = launch_flops / (launch_ms * 1e-3) / 1e12
-        roofline = {"bound": "tensor", "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
-                    "frac": achieved / peak_tf, "traffic": traffic,
-                    "peak_source": f"{peak_src} {'sustained' if long_step else 'burst'} bf16 dense",
-                    "kernel": "lowbit_gemm_kernel (each timed launch is one lowbit_gemm call: X conversion "
-                              "pass + GEMM kernel)", "launches_timed": len(per),
+        # Each per-launch figure comes from short back-to-back replays of one shape (a few ms),
+        # a kernel timed on its own: the burst peak applies.
+        achieved = launch_flops / (gemm_ms * 1e-3) / 1e12
+        call = launch_flops / (launch_ms * 1e-3) / 1e12
+        roofline = {"bound": "tensor", "achieved": achieved, "peak": burst, "unit": "TFLOP/s",
+                    "frac": achieved / burst, "traffic": traffic,
+                    "peak_source": f"{peak_src} burst bf16 dense (kernels timed in short back-to-back replays)",
+                    "kernel": "lowbit_gemm_kernel (GEMM kernel alone: the X conversion's share is taken out)",
+                    "us_per_launch": gemm_ms * 1e3, "launches_timed": launches_timed,
                     "algorithmic_gflop_per_launch": launch_flops / 1e9,
                     "algorithmic_mb_per_launch": launch_bytes / 1e6,
-                    "frac_of_burst_peak": achieved / peaks.get("bf16_tflops", peak_tf)}
+                    "call": {"what": "one lowbit_gemm call = X conversion pass + GEMM kernel",
+                             "achieved": call, "frac": call / burst, "us_per_launch": launch_ms * 1e3,
+                             "x_conversion_us_per_launch": conv_ms * 1e3},
+                    "step_frac_of_burst_peak": (flops / (ms_step * 1e-3) / 1e12) / burst}
+        if copies > 1:
+            roofline["weight_copies_rotated"] = copies
 
     if rank == 0:
         spec0 = specs[0]
@@ -515,20 +555,36 @@ def run_lowbit(args, specs, workload):
             line["config"]["ms_per_4_steps"] = 4 * ms_step
         print(json.dumps(line), flush=True)
         if args.per_shape:
-            agg = {}
-            for sp, ms in per:
-                k = (sp.M, sp.K, sp.N)
-                agg.setdefault(k, []).append(ms)
-            for k, v in sorted(agg.items()):
-                m, kk, n = k
-                t = statistics.median(v)
-                print(f"# shape M={m} K={kk} N={n}: {t * 1e3:.1f} us, {2 * m * kk * n / t / 1e9:.1f} TFLOP/s",
+            for (m, kk, n), (t_call, t_gemm, t_conv, reps) in sorted(shape_times.items()):
+                f = 2 * m * kk * n
+                sp = next(x for x in specs if (x.M, x.K, x.N) == (m, kk, n))
+                print(f"# shape M={m} K={kk} N={n}: call {t_call * 1e3:.2f} us ({f / t_call / 1e9:.1f} TFLOP/s, "
+                      f"{sp.algorithmic_bytes() / t_call / 1e6:.0f} GB/s); GEMM kernel {t_gemm * 1e3:.2f} us "
+                      f"({f / t_gemm / 1e9:.1f} TFLOP/s); X conversion {t_conv * 1e3:.2f} us; {reps} per graph",
                       file=sys.stderr)
     del graphs, items, descs
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def relaunch_under_torchrun(gpus: int, argv) -> int:
+    """Run this script as `gpus` ranks of one node (torchrun, rendezvous on 127.0.0.1) and return
+    their exit status: `--gpus N` outside torchrun never times one GPU under an N-GPU label."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={gpus}",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__), *argv]
+    return subprocess.call(cmd)
+
+
+def check_world(gpus: int, world: int) -> None:
+    """The ranks that run must be the GPUs the line will report."""
+    if world != gpus:
+        raise SystemExit(f"bench.py: --gpus {gpus} but {world} ranks were launched")
 
 
 def main():
@@ -546,6 +602,13 @@ def main():
                                                       "(profiling one shape); default all")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)   # at least 3 untimed warm-up steps
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        if args.impl == "lowbit":
+            import torch
+            if torch.cuda.device_count() < args.gpus:
+                raise SystemExit(f"bench.py: --gpus {args.gpus} but {torch.cuda.device_count()} GPUs are visible")
+        return relaunch_under_torchrun(args.gpus, sys.argv[1:])
+    check_world(args.gpus, int(os.environ.get("WORLD_SIZE", "1")))
     specs = synth.WORKLOADS[args.workload]
     if args.only_linear:
         specs = [specs[int(i)] for i in args.only_linear.split(",")]

@@ -1,9 +1,11 @@
 """Build liblowbit.so (the CUDA library) in-tree with nvcc for sm_100a.
 
-    python -m bit_weight_only_w2_b200.build [--force]
+    python -m bit_weight_only_w2_b200.build [--force] [--debug]
 
 Objects go to ``_build/`` at the repository root; the shared library is written next to this
-file so the Python binding (and a copy of the tree on another machine) finds it.
+file so the Python binding (and a copy of the tree on another machine) finds it. ``--debug``
+builds liblowbit_debug.so instead: the same sources with device-side index checks
+(LOWBIT_DEBUG_CHECKS), objects in ``_build/debug/``.
 """
 from __future__ import annotations
 
@@ -18,6 +20,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "liblowbit.so")
+DEBUG_LIB = os.path.join(PKG, "liblowbit_debug.so")
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -42,8 +45,8 @@ def _stale(target, inputs):
     return any(os.path.getmtime(i) > t for i in inputs)
 
 
-def _compile(src, obj, verbose):
-    cmd = [NVCC, *ARCH, *FLAGS, "-c", src, "-o", obj]
+def _compile(src, obj, verbose, extra=()):
+    cmd = [NVCC, *ARCH, *FLAGS, *extra, "-c", src, "-o", obj]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     r = subprocess.run(cmd, capture_output=True, text=True)
@@ -52,28 +55,31 @@ def _compile(src, obj, verbose):
     return r.stderr
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
+    out_dir = os.path.join(BUILD, "debug") if debug else BUILD
+    lib = DEBUG_LIB if debug else LIB
+    extra = ("-DLOWBIT_DEBUG_CHECKS",) if debug else ()
+    os.makedirs(out_dir, exist_ok=True)
     deps = _deps()
     objs = []
     jobs = []
     for src in sources():
-        obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(out_dir, os.path.basename(src)[:-3] + ".o")
         objs.append(obj)
         if force or _stale(obj, [src, *deps]):
             jobs.append((src, obj))
     if jobs:
         with cf.ThreadPoolExecutor(max_workers=max(1, min(len(jobs), os.cpu_count() or 1))) as ex:
-            for log in ex.map(lambda j: _compile(j[0], j[1], verbose), jobs):
+            for log in ex.map(lambda j: _compile(j[0], j[1], verbose, extra), jobs):
                 if verbose and log:
                     sys.stderr.write(log)
-    if force or jobs or _stale(LIB, objs):
-        tmp = LIB + f".tmp{os.getpid()}"
+    if force or jobs or _stale(lib, objs):
+        tmp = lib + f".tmp{os.getpid()}"
         cmd = [NVCC, *ARCH, "-shared", "-o", tmp, *objs, "-Xcompiler", "-fvisibility=hidden"]
         subprocess.check_call(cmd)
-        os.replace(tmp, LIB)
-    return LIB
+        os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv, debug="--debug" in sys.argv))

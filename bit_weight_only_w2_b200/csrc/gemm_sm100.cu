@@ -178,10 +178,15 @@ __device__ __forceinline__ void decode_word_b2(uint32_t v, uint32_t s2, uint32_t
 }
 
 // uint4: the nibbles of a pair, left at bit 4j of each half (j <= 1), OR-ed into fp16 1024.0
-// give 1024 + q * 16^j exactly; one FMA recovers q exactly and a second computes
-// q * s + (-z * s), rounded once to fp16. c2 = fp16x2(-z * s) of the group. Word w of the half
-// (block w / 4, word q = w % 4 of it): pair c goes to out[16 * (w / 4) + 4c + q].
-__device__ __forceinline__ void decode_word_b4(uint32_t v, uint32_t s2, uint32_t c2, uint32_t* out, int w) {
+// give 1024 + q * 16^j exactly, and one fp16x2 FMA recovers q exactly. Each weight is then
+// (q - z) * s = q * s + cz with cz = -z * s in fp32 (exact: the product of two fp16 values has
+// at most 22 significant bits), formed by one mixed-precision FMA (q * s is exact as well, so
+// the only fp32 rounding is below 2^-24 relative) and rounded to fp16 once. A code equal or
+// next to its zero point thus keeps the full fp16 precision of the small difference (q - z) * s;
+// rounding -z * s to fp16 first would cost up to 2^-11 |z * s| per weight, which is most of
+// such a weight. Word w of the half (block w / 4, word q = w % 4 of it): pair c goes to
+// out[16 * (w / 4) + 4c + q].
+__device__ __forceinline__ void decode_word_b4(uint32_t v, uint16_t s, float cz, uint32_t* out, int w) {
     constexpr uint32_t kMagic = 0x64006400u;
     constexpr uint32_t kMul[2] = {0x3C003C00u, 0x2C002C00u};   // 1, 1/16
     constexpr uint32_t kAdd[2] = {0xE400E400u, 0xD400D400u};   // -1024, -64
@@ -191,7 +196,9 @@ __device__ __forceinline__ void decode_word_b4(uint32_t v, uint32_t s2, uint32_t
         const int j = c & 1;
         const uint32_t e = and_or(v >> shift, 0x000F000Fu << (4 * j), kMagic);
         const uint32_t q = f16x2_fma(e, kMul[j], kAdd[j]);
-        out[16 * (w >> 2) + 4 * c + (w & 3)] = f16x2_fma(q, s2, c2);
+        float lo, hi;
+        fma_f16x2_f32(q, s, cz, lo, hi);
+        out[16 * (w >> 2) + 4 * c + (w & 3)] = pack_f16x2(lo, hi);
     }
 }
 
@@ -415,7 +422,8 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT>::kThreads, Cfg<BITS, GS, BT>
                 const uint8_t* st = wring + s * C::kWStageBytes;
                 // --- this row's packed words and scales (rows past the tile decode to zero)
                 uint32_t words[kHalvesPerPart][C::kWordsPerRow / 2];
-                uint32_t s2[kHalvesPerPart], c2[kHalvesPerPart];
+                uint32_t s2[kHalvesPerPart];
+                float cz[kHalvesPerPart];
                 const uint8_t* wrow = st + C::kWOff + row * C::kWRowBytes;
 #pragma unroll
                 for (int hh = 0; hh < kHalvesPerPart; ++hh) {
@@ -424,7 +432,7 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT>::kThreads, Cfg<BITS, GS, BT>
 #pragma unroll
                     for (int w = 0; w < C::kWordsPerRow / 2; ++w) words[hh][w] = 0;
                     s2[hh] = 0;
-                    c2[hh] = 0;
+                    cz[hh] = 0.f;
                     if (row_ok) {
                         if (BITS == 1) {
                             const uint2 v = *reinterpret_cast<const uint2*>(wrow + h * 8);
@@ -446,12 +454,10 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT>::kThreads, Cfg<BITS, GS, BT>
                         const uint16_t* srow = reinterpret_cast<const uint16_t*>(st + C::kSOff) + gi * kBlockN;
                         const uint32_t sb = srow[row];
                         s2[hh] = sb | (sb << 16);
-                        if (BITS == 4) {
+                        if (BITS == 4) {   // -z * s, exact in fp32
                             const __half* zrow = reinterpret_cast<const __half*>(st + C::kZOff) + gi * kBlockN;
-                            const float cz = -__half2float(zrow[row]) *
-                                             __half2float(__ushort_as_half(static_cast<unsigned short>(sb)));
-                            const uint32_t cb = __half_as_ushort(__float2half_rn(cz));
-                            c2[hh] = cb | (cb << 16);
+                            cz[hh] = -__half2float(zrow[row]) *
+                                     __half2float(__ushort_as_half(static_cast<unsigned short>(sb)));
                         }
                     }
                 }
@@ -474,9 +480,11 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT>::kThreads, Cfg<BITS, GS, BT>
                         for (int w = 0; w < 4; ++w) decode_word_b2(words[hh][w], s2[hh], out, w);
                     } else {
 #pragma unroll
-                        for (int w = 0; w < 8; ++w) decode_word_b4(words[hh][w], s2[hh], c2[hh], out, w);
+                        for (int w = 0; w < 8; ++w)
+                            decode_word_b4(words[hh][w], static_cast<uint16_t>(s2[hh]), cz[hh], out, w);
                     }
-                    tmem_st32(lane_base + C::kACol0 + a * 64 + h * 32, out);
+                    if (dcheck(C::kACol0 + a * 64 + h * 32 + 32 <= C::kTmemCols, status))
+                        tmem_st32(lane_base + C::kACol0 + a * 64 + h * 32, out);
                 }
                 tmem_wait_st();
                 tc_fence_before();
@@ -508,7 +516,7 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT>::kThreads, Cfg<BITS, GS, BT>
 #pragma unroll
             for (int ci = 0; ci < kChunks; ++ci) {
                 const int mj = m0 + ci * kChunk + lane;
-                mul[ci] = (!split && lane < kChunk && mj < p.M) ? p.rowmul[mj] : 1.0f;
+                mul[ci] = (!split && lane < kChunk && mj < p.M && dcheck(mj >= 0, status)) ? p.rowmul[mj] : 1.0f;
             }
             if (!__all_sync(0xffffffffu, mbar_wait(&accfull[b], acc_ph, abort_flag, status))) break;
             tc_fence_after();
@@ -549,7 +557,8 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT>::kThreads, Cfg<BITS, GS, BT>
                     const uint32_t other = __shfl_xor_sync(0xffffffffu, mine, 1);
                     const uint32_t outw = even ? __byte_perm(mine, other, 0x5410) : __byte_perm(other, mine, 0x7632);
                     const int m = m0 + j + (even ? 0 : 1);
-                    if (pair_ok && m < p.M)
+                    if (pair_ok && m < p.M &&
+                        dcheck(m >= 0 && n_pair >= 0 && n_pair + 1 < p.N && (n_pair & 1) == 0, status))
                         *reinterpret_cast<uint32_t*>(p.Y + static_cast<size_t>(m) * p.N + n_pair) = outw;
                 }
             } else {
@@ -644,7 +653,7 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT>::kThreads, Cfg<BITS, GS, BT>
 #pragma unroll
                         for (int j = 0; j < 4; ++j) {
                             const int m = m0 + cc + j;
-                            if (m < p.M)
+                            if (m < p.M && dcheck(m >= 0 && n >= 0 && n < p.N && cc + j < BT, status))
                                 p.Y[static_cast<size_t>(m) * p.N + n] = __float2bfloat16_rn(a4[j] * fac[cc + j]);
                         }
                     }
@@ -749,6 +758,7 @@ lowbit_status launch_convert_x(const GemmProblem& g, cudaStream_t stream) {
     ccfg.attrs = cattr;
     ccfg.numAttrs = 1;
     const int K8 = static_cast<int>(g.K / 8);
+    if (take_injected_failure(kInjectLaunch)) return LOWBIT_ERR_CUDA;
     const uint4* x = static_cast<const uint4*>(g.X);
     uint4* xh = static_cast<uint4*>(g.workspace);
     float* rm = reinterpret_cast<float*>(static_cast<uint8_t*>(g.workspace) + ws.rowmul_offset);
@@ -780,6 +790,21 @@ lowbit_status selftest_bounded_wait(long long limit_cycles, cudaStream_t stream)
     return cudaGetLastError() == cudaSuccess ? LOWBIT_OK : LOWBIT_ERR_CUDA;
 }
 
+// One thread asks to store one element past a one-element array. The store happens only when
+// the index is in range, so nothing is ever written out of bounds; in debug builds the index
+// check in front of it records the failure in the status word, as the GEMM kernels' checks do.
+__device__ unsigned g_selftest_cell[1];
+__global__ void index_check_selftest_kernel(int index) {
+    const bool ok = index >= 0 && index < 1;
+    if (dcheck(ok, &g_device_status) && ok) g_selftest_cell[index] = 1u;
+}
+
+lowbit_status selftest_index_check(cudaStream_t stream) {
+    if (!kDebugChecks) return LOWBIT_ERR_UNSUPPORTED;
+    index_check_selftest_kernel<<<1, 1, 0, stream>>>(1);
+    return cudaGetLastError() == cudaSuccess ? LOWBIT_OK : LOWBIT_ERR_CUDA;
+}
+
 // ---------------------------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------------------------
@@ -805,6 +830,7 @@ struct MapKey {
 
 bool encode_cached(CUtensorMap* map, CUtensorMapDataType dtype, int rank, const void* base, const uint64_t* dims,
                    const uint64_t* strides, const uint32_t* box, CUtensorMapSwizzle swz) {
+    if (take_injected_failure(kInjectEncode)) return false;
     constexpr int kSlots = 1024;
     struct Slot {
         bool used;
@@ -951,7 +977,7 @@ int num_sms() {
 namespace {
 
 template <int BITS, int GS, int BT>
-lowbit_status launch(const GemmProblem& g, int rows, int ksplit_request, cudaStream_t stream) {
+lowbit_status launch(const GemmProblem& g, int rows, int ksplit_request, cudaStream_t stream, bool convert_x) {
     using C = Cfg<BITS, GS, BT>;
     auto kernel = lowbit_gemm_kernel<BITS, GS, BT>;
     // the shared-memory opt-in is per device: one bit per device that has it
@@ -1022,7 +1048,7 @@ lowbit_status launch(const GemmProblem& g, int rows, int ksplit_request, cudaStr
 
     // X -> fp16 copy in the workspace, then the GEMM; both launched as programmatic dependents
     // of whatever precedes them on the stream.
-    if (launch_convert_x(g, stream) != LOWBIT_OK) return LOWBIT_ERR_CUDA;
+    if (convert_x && launch_convert_x(g, stream) != LOWBIT_OK) return LOWBIT_ERR_CUDA;
 
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attrs[2];
@@ -1046,6 +1072,7 @@ lowbit_status launch(const GemmProblem& g, int rows, int ksplit_request, cudaStr
     cfg.stream = stream;
     cfg.attrs = attrs;
     cfg.numAttrs = na;
+    if (take_injected_failure(kInjectLaunch)) return LOWBIT_ERR_CUDA;
     cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, mx, mw, ms, mz, p);
     return e == cudaSuccess ? LOWBIT_OK : LOWBIT_ERR_CUDA;
 }
@@ -1062,13 +1089,13 @@ int pick_bt(int64_t M) {
 int ctas_per_sm_for(int bt) { return bt <= 64 ? 2 : 1; }
 
 template <int BITS, int GS>
-lowbit_status launch_bits_gs(const GemmProblem& g, int bt, int rows, int ksplit, cudaStream_t s) {
+lowbit_status launch_bits_gs(const GemmProblem& g, int bt, int rows, int ksplit, cudaStream_t s, bool cx) {
     switch (bt) {
-        case 16: return launch<BITS, GS, 16>(g, rows, ksplit, s);
-        case 32: return launch<BITS, GS, 32>(g, rows, ksplit, s);
-        case 64: return launch<BITS, GS, 64>(g, rows, ksplit, s);
-        case 128: return launch<BITS, GS, 128>(g, rows, ksplit, s);
-        case 256: return launch<BITS, GS, 256>(g, rows, ksplit, s);
+        case 16: return launch<BITS, GS, 16>(g, rows, ksplit, s, cx);
+        case 32: return launch<BITS, GS, 32>(g, rows, ksplit, s, cx);
+        case 64: return launch<BITS, GS, 64>(g, rows, ksplit, s, cx);
+        case 128: return launch<BITS, GS, 128>(g, rows, ksplit, s, cx);
+        case 256: return launch<BITS, GS, 256>(g, rows, ksplit, s, cx);
         default: return LOWBIT_ERR_UNSUPPORTED;
     }
 }
@@ -1081,11 +1108,15 @@ lowbit_status launch_bits_gs(const GemmProblem& g, int bt, int rows, int ksplit,
 //     tiles with K split over a cluster, whichever reads fewer X bytes per weight byte;
 //   * few tiles otherwise: 128-row tiles with K split over a cluster;
 //   * many tiles: 128-row tiles on a persistent grid.
+bool uses_x_copy(const GemmProblem& g) { return !smallm_supported(g); }
+
 lowbit_status gemm_launch(const GemmProblem& g, int force_bt, int force_rows, int force_split,
-                          cudaStream_t stream) {
-    // tile_tokens == 1 selects the small-M warp-MMA kernel; automatic choice for M <= 16
-    if (force_bt == 1) return smallm_launch(g, force_rows, force_split, stream);
-    if (!force_bt && !force_rows && !force_split && smallm_supported(g)) return smallm_launch(g, 0, 0, stream);
+                          cudaStream_t stream, bool convert_x) {
+    // tile_tokens == 1 selects the small-M warp-MMA kernel with X as the 16-row operand, 8 the
+    // one with weights as the 16-row operand (M <= 8); automatic: 8 for M <= 8, else 1 up to 16
+    if (force_bt == 1 || force_bt == 8) return smallm_launch(g, force_rows, force_split, force_bt == 8, stream);
+    if (!force_bt && !force_rows && !force_split && smallm_supported(g))
+        return smallm_launch(g, 0, 0, g.M <= 8, stream);
     const int bt = force_bt ? force_bt : pick_bt(g.M);
     const int sms = num_sms();
     const int64_t num_kb = (g.K + kBlockK - 1) / kBlockK;
@@ -1115,28 +1146,42 @@ lowbit_status gemm_launch(const GemmProblem& g, int force_bt, int force_rows, in
     if (!ksplit) ksplit = 1;
     if (rows < 8 || rows > kBlockN || rows % 8) return LOWBIT_ERR_UNSUPPORTED;   // (ksplit -1: automatic)
     switch (g.bits * 1000 + g.group_size) {
-        case 1064: return launch_bits_gs<1, 64>(g, bt, rows, ksplit, stream);
-        case 1128: return launch_bits_gs<1, 128>(g, bt, rows, ksplit, stream);
-        case 2064: return launch_bits_gs<2, 64>(g, bt, rows, ksplit, stream);
-        case 2128: return launch_bits_gs<2, 128>(g, bt, rows, ksplit, stream);
-        case 4064: return launch_bits_gs<4, 64>(g, bt, rows, ksplit, stream);
-        case 4128: return launch_bits_gs<4, 128>(g, bt, rows, ksplit, stream);
+        case 1064: return launch_bits_gs<1, 64>(g, bt, rows, ksplit, stream, convert_x);
+        case 1128: return launch_bits_gs<1, 128>(g, bt, rows, ksplit, stream, convert_x);
+        case 2064: return launch_bits_gs<2, 64>(g, bt, rows, ksplit, stream, convert_x);
+        case 2128: return launch_bits_gs<2, 128>(g, bt, rows, ksplit, stream, convert_x);
+        case 4064: return launch_bits_gs<4, 64>(g, bt, rows, ksplit, stream, convert_x);
+        case 4128: return launch_bits_gs<4, 128>(g, bt, rows, ksplit, stream, convert_x);
         default: return LOWBIT_ERR_UNSUPPORTED;
     }
 }
 
 unsigned* device_status_address() {
     constexpr int kMaxDevices = 64;
-    static unsigned* ptrs[kMaxDevices] = {};
+    static std::atomic<unsigned*> ptrs[kMaxDevices];
+    static std::mutex mu;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-    if (!ptrs[dev]) {
+    unsigned* p = ptrs[dev].load(std::memory_order_acquire);
+    if (p) return p;
+    std::lock_guard<std::mutex> lock(mu);
+    p = ptrs[dev].load(std::memory_order_relaxed);
+    if (!p) {
         void* ptr = nullptr;
         if (cudaGetSymbolAddress(&ptr, g_device_status) != cudaSuccess) return nullptr;
-        ptrs[dev] = static_cast<unsigned*>(ptr);
+        p = static_cast<unsigned*>(ptr);
+        ptrs[dev].store(p, std::memory_order_release);
     }
-    return ptrs[dev];
+    return p;
 }
+
+namespace {
+lowbit_status status_of_word(unsigned v) {
+    if (v & kDevErrTimeout) return LOWBIT_ERR_TIMEOUT;
+    if (v & kDevErrCheck) return LOWBIT_ERR_DEVICE_CHECK;
+    return LOWBIT_OK;
+}
+}  // namespace
 
 lowbit_status read_device_status(int clear) {
     unsigned v = 0;
@@ -1146,7 +1191,20 @@ lowbit_status read_device_status(int clear) {
         const unsigned zero = 0;
         if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(zero)) != cudaSuccess) return LOWBIT_ERR_CUDA;
     }
-    return (v & kDevErrTimeout) ? LOWBIT_ERR_TIMEOUT : LOWBIT_OK;
+    return status_of_word(v);
+}
+
+// Stream-ordered read and clear: the copy of the word and the clearing store are queued on
+// `stream`, so only the work queued there before them is waited for.
+lowbit_status read_stream_status(cudaStream_t stream) {
+    unsigned* word = device_status_address();
+    if (!word) return LOWBIT_ERR_CUDA;
+    unsigned v = 0;
+    if (cudaMemcpyAsync(&v, word, sizeof(v), cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
+        cudaMemsetAsync(word, 0, sizeof(unsigned), stream) != cudaSuccess ||
+        cudaStreamSynchronize(stream) != cudaSuccess)
+        return LOWBIT_ERR_CUDA;
+    return status_of_word(v);
 }
 
 }  // namespace lowbit

@@ -6,6 +6,8 @@
 #include <cstdlib>
 #include <atomic>
 #include <mutex>
+#include <utility>
+#include <vector>
 
 #include "lowbit_internal.h"
 
@@ -50,6 +52,17 @@ lowbit_status check_device() {
     return ok ? LOWBIT_OK : LOWBIT_ERR_UNSUPPORTED_DEVICE;
 }
 
+namespace {
+std::atomic<int> g_injected{0};   // InjectKind bits still to be consumed
+}  // namespace
+
+bool take_injected_failure(int kind) {
+    int cur = g_injected.load(std::memory_order_relaxed);
+    while (cur & kind)
+        if (g_injected.compare_exchange_weak(cur, cur & ~kind, std::memory_order_acq_rel)) return true;
+    return false;
+}
+
 lowbit_status validate_gemm(const GemmProblem& g) {
     if (!valid_bits(g.bits)) return LOWBIT_ERR_INVALID_ARG;
     if (g.M < 0 || g.N < 0 || g.K <= 0 || g.group_size <= 0) return LOWBIT_ERR_INVALID_ARG;
@@ -87,6 +100,7 @@ LOWBIT_API const char* lowbit_status_string(lowbit_status s) {
         case LOWBIT_ERR_TIMEOUT: return "LOWBIT_ERR_TIMEOUT";
         case LOWBIT_ERR_CUDA: return "LOWBIT_ERR_CUDA";
         case LOWBIT_ERR_WORKSPACE: return "LOWBIT_ERR_WORKSPACE";
+        case LOWBIT_ERR_DEVICE_CHECK: return "LOWBIT_ERR_DEVICE_CHECK";
     }
     return "LOWBIT_ERR_UNKNOWN";
 }
@@ -163,10 +177,11 @@ LOWBIT_API lowbit_status lowbit_gemm_ex(int64_t M, int64_t N, int64_t K, int bit
     const GemmProblem g = make_problem(M, N, K, bits, group_size, X, Wp, scales, zeros, Y, workspace, workspace_bytes);
     lowbit_status st = validate_gemm(g);
     if (st != LOWBIT_OK || M == 0 || N == 0) return st;
-    if (tile_tokens != 0 && tile_tokens != 1 && tile_tokens != 16 && tile_tokens != 32 && tile_tokens != 64 &&
-        tile_tokens != 128 && tile_tokens != 256)
+    if (tile_tokens != 0 && tile_tokens != 1 && tile_tokens != 8 && tile_tokens != 16 && tile_tokens != 32 &&
+        tile_tokens != 64 && tile_tokens != 128 && tile_tokens != 256)
         return LOWBIT_ERR_UNSUPPORTED;
-    if (tile_tokens == 1 && M > 16) return LOWBIT_ERR_UNSUPPORTED;
+    if ((tile_tokens == 1 && M > 16) || (tile_tokens == 8 && M > 8)) return LOWBIT_ERR_UNSUPPORTED;
+    if (tile_tokens == 8 && tile_rows % 16 != 0) return LOWBIT_ERR_UNSUPPORTED;
     if (ksplit < 0 || ksplit > 8) return LOWBIT_ERR_UNSUPPORTED;
     if (tile_rows < 0 || tile_rows > 128 || tile_rows % 8 != 0) return LOWBIT_ERR_UNSUPPORTED;
     if ((st = check_device()) != LOWBIT_OK) return st;
@@ -185,18 +200,68 @@ LOWBIT_API lowbit_status lowbit_gemm_batch(const lowbit_gemm_desc* descs, int co
     if (count == 0) return LOWBIT_OK;
     lowbit_status st = check_device();
     if (st != LOWBIT_OK) return st;
+    // The fp16 copy of X in the workspace is reused by the next linear that reads the same X
+    // (same pointer, M and K) when no output written since the copy was made overlaps that X:
+    // e.g. separate Q, K and V projections of one input convert it once.
+    const void* copied_x = nullptr;
+    int64_t copied_m = -1, copied_k = -1;
+    std::vector<std::pair<uintptr_t, uintptr_t>> written;   // Y byte ranges since the copy
     for (int i = 0; i < count; ++i) {
         const lowbit_gemm_desc& d = descs[i];
         if (d.M == 0 || d.N == 0) continue;
-        st = gemm_launch(make_problem(d.M, d.N, d.K, d.bits, d.group_size, d.X, d.Wp, d.scales, d.zeros, d.Y,
-                                      workspace, workspace_bytes),
-                         0, 0, 0, static_cast<cudaStream_t>(stream));
+        const GemmProblem g = make_problem(d.M, d.N, d.K, d.bits, d.group_size, d.X, d.Wp, d.scales, d.zeros, d.Y,
+                                           workspace, workspace_bytes);
+        bool convert = true;
+        if (uses_x_copy(g)) {
+            const uintptr_t x0 = reinterpret_cast<uintptr_t>(d.X), x1 = x0 + static_cast<uintptr_t>(d.M * d.K * 2);
+            bool clean = copied_x == d.X && copied_m == d.M && copied_k == d.K;
+            for (size_t j = 0; clean && j < written.size(); ++j)
+                if (written[j].first < x1 && x0 < written[j].second) clean = false;
+            convert = !clean;
+        }
+        st = gemm_launch(g, 0, 0, 0, static_cast<cudaStream_t>(stream), convert);
         if (st != LOWBIT_OK) return st;
+        if (uses_x_copy(g) && convert) {
+            copied_x = d.X;
+            copied_m = d.M;
+            copied_k = d.K;
+            written.clear();
+        }
+        const uintptr_t y0 = reinterpret_cast<uintptr_t>(d.Y);
+        written.emplace_back(y0, y0 + static_cast<uintptr_t>(d.M * d.N * 2));
     }
     return LOWBIT_OK;
 }
 
 LOWBIT_API lowbit_status lowbit_device_status(int clear) { return read_device_status(clear); }
+
+LOWBIT_API lowbit_status lowbit_last_device_status(void* stream) {
+    const lowbit_status st = check_device();
+    if (st != LOWBIT_OK) return st;
+    return read_stream_status(static_cast<cudaStream_t>(stream));
+}
+
+LOWBIT_API lowbit_status lowbit_test_fail_next(int what) {
+    if (what < 0 || what > (kInjectEncode | kInjectLaunch)) return LOWBIT_ERR_INVALID_ARG;
+    if (what == 0) g_injected.store(0, std::memory_order_release);
+    else g_injected.fetch_or(what, std::memory_order_acq_rel);
+    return LOWBIT_OK;
+}
+
+LOWBIT_API int lowbit_debug_checks_enabled(void) {
+#ifdef LOWBIT_DEBUG_CHECKS
+    return 1;
+#else
+    return 0;
+#endif
+}
+
+LOWBIT_API lowbit_status lowbit_selftest_index_check(void* stream) {
+    if (!lowbit_debug_checks_enabled()) return LOWBIT_ERR_UNSUPPORTED;
+    const lowbit_status st = check_device();
+    if (st != LOWBIT_OK) return st;
+    return selftest_index_check(static_cast<cudaStream_t>(stream));
+}
 
 LOWBIT_API lowbit_status lowbit_selftest_bounded_wait(long long limit_cycles, void* stream) {
     if (limit_cycles <= 0) return LOWBIT_ERR_INVALID_ARG;

@@ -38,8 +38,14 @@ lowbit_status validate_gemm(const GemmProblem& g);
 
 // Launches the X conversion and the GEMM kernel for a validated problem. force_bt (tokens per
 // tile), force_rows (weight rows per tile) and force_split (K slices): 0 = automatic.
+// convert_x = false skips the conversion when the workspace already holds this X's fp16 copy
+// and row factors (a batch whose previous linear read the same, unchanged X).
 lowbit_status gemm_launch(const GemmProblem& g, int force_bt, int force_rows, int force_split,
-                          cudaStream_t stream);
+                          cudaStream_t stream, bool convert_x = true);
+
+// True if the problem runs on the tensor-memory kernel (and so through the X conversion pass)
+// when its configuration is chosen automatically.
+bool uses_x_copy(const GemmProblem& g);
 
 // Launches the X -> fp16 conversion pass into the problem's workspace (programmatic dependent
 // launch). The GEMM kernels read its output.
@@ -47,9 +53,11 @@ lowbit_status launch_convert_x(const GemmProblem& g, cudaStream_t stream);
 
 // Small-M GEMM (M <= 16) on warp-level bf16 tensor-core MMAs, reading X directly (no
 // conversion pass, no workspace). rows (weight rows per CTA, multiple of 8, <= 128) and ksplit
-// (K slices per cluster, <= 8): 0 = automatic. smallm_supported: whether the shape fits it.
+// (K slices per cluster, <= 8): 0 = automatic. swap: weights as the MMA's 16-row operand and up
+// to 8 tokens as its n8 operand (M <= 8; rows a multiple of 16). smallm_supported: whether the
+// shape fits the kernel at all.
 bool smallm_supported(const GemmProblem& g);
-lowbit_status smallm_launch(const GemmProblem& g, int rows, int ksplit, cudaStream_t stream);
+lowbit_status smallm_launch(const GemmProblem& g, int rows, int ksplit, bool swap, cudaStream_t stream);
 
 // Device address of the current device's status word (nullptr on failure).
 unsigned* device_status_address();
@@ -65,6 +73,9 @@ bool make_map_3d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, 
 // Reads (and optionally clears) the device status word. Synchronises the device.
 lowbit_status read_device_status(int clear);
 
+// Reads and clears the device status word in the order of `stream`, waiting for that stream only.
+lowbit_status read_stream_status(cudaStream_t stream);
+
 // Packing kernels (synchronous on `stream`); `bad` receives the number of invalid codes.
 lowbit_status pack_launch(const int8_t* codes, int64_t N, int64_t K, int bits, uint32_t* packed,
                           cudaStream_t stream, unsigned long long* bad);
@@ -74,7 +85,15 @@ lowbit_status unpack_launch(const uint32_t* packed, int64_t N, int64_t K, int bi
 // Launches the bounded-wait self-test kernel.
 lowbit_status selftest_bounded_wait(long long limit_cycles, cudaStream_t stream);
 
+// Launches the index-check self-test kernel (debug builds; else LOWBIT_ERR_UNSUPPORTED).
+lowbit_status selftest_index_check(cudaStream_t stream);
+
 // True when the current device can run the sm_100a kernels.
 lowbit_status check_device();
+
+// Failure injection for tests of the error paths (lowbit_test_fail_next): true, once, if a
+// failure of `kind` was requested; the call site then reports it as the real failure would.
+enum InjectKind { kInjectEncode = 1, kInjectLaunch = 2 };
+bool take_injected_failure(int kind);
 
 }  // namespace lowbit

@@ -12,7 +12,22 @@ namespace lowbit {
 // A wait that has not completed after this many SM clocks (about 2 s at 1.9 GHz) gives up,
 // records LOWBIT_DEVERR_TIMEOUT in the device status word and raises the CTA's abort flag.
 constexpr long long kWaitLimitCycles = 4000000000LL;
-constexpr unsigned kDevErrTimeout = 1u;
+constexpr unsigned kDevErrTimeout = 1u;   // a bounded wait gave up
+constexpr unsigned kDevErrCheck = 2u;     // a device-side index check failed (debug builds)
+
+// Device-side index checks of the debug build (LOWBIT_DEBUG_CHECKS): dcheck(ok, word) records
+// kDevErrCheck in the status word when `ok` is false and returns `ok`, so the caller skips the
+// access instead of trapping; release builds compile the checks away.
+#ifdef LOWBIT_DEBUG_CHECKS
+constexpr bool kDebugChecks = true;
+__device__ __forceinline__ bool dcheck(bool ok, unsigned* status_word) {
+    if (!ok) atomicOr(status_word, kDevErrCheck);
+    return ok;
+}
+#else
+constexpr bool kDebugChecks = false;
+__device__ __forceinline__ bool dcheck(bool, unsigned*) { return true; }
+#endif
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -247,6 +262,16 @@ __device__ __forceinline__ uint32_t f16x2_mul(uint32_t a, uint32_t b) {
     uint32_t d;
     asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
     return d;
+}
+// Mixed-precision FMA on both halves of an fp16x2 value a: lo = a.lo * b + c, hi = a.hi * b + c,
+// with b fp16 (bit pattern), c and the results fp32, each rounded once to fp32.
+__device__ __forceinline__ void fma_f16x2_f32(uint32_t a, uint16_t b, float c, float& lo, float& hi) {
+    asm("{\n\t.reg .b16 al, ah;\n\t"
+        "mov.b32 {al, ah}, %2;\n\t"
+        "fma.rn.f32.f16 %0, al, %3, %4;\n\t"
+        "fma.rn.f32.f16 %1, ah, %3, %4;\n\t}\n"
+        : "=f"(lo), "=f"(hi)
+        : "r"(a), "h"(b), "f"(c));
 }
 // fp16x2 with `lo` in the low half, both rounded to nearest even.
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {

@@ -1,4 +1,5 @@
-// Host side of the small-M kernel (smallm_kernel.cuh): tile choice, tensor maps and launch.
+// Host side of the small-M kernel (smallm_kernel.cuh): orientation, tile choice, tensor maps and
+// launch.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -11,11 +12,11 @@ namespace lowbit {
 namespace smallm {
 namespace {
 
-const void* kernel_for(int bits, int gs, int noct) {
+const void* kernel_for(int bits, int gs, int noct, bool swap) {
     switch (bits) {
-        case 1: return kernel_b1(gs, noct);
-        case 2: return kernel_b2(gs, noct);
-        case 4: return kernel_b4(gs, noct);
+        case 1: return kernel_b1(gs, noct, swap);
+        case 2: return kernel_b2(gs, noct, swap);
+        case 4: return kernel_b4(gs, noct, swap);
         default: return nullptr;
     }
 }
@@ -29,7 +30,7 @@ bool prepare(const void* fn) {
         const void* fn;
         int dev;
     };
-    static Done done[8 * 3 * 2 * kMaxOct];
+    static Done done[8 * 3 * 2 * (kMaxOct + kMaxOct / 2)];
     static int used = 0;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return false;
@@ -44,16 +45,16 @@ bool prepare(const void* fn) {
 // Clusters of `ks` CTAs that fit on the current device at once (one CTA per SM), cached per
 // device and entry point family (all octet counts of a format share the occupancy of one CTA
 // per SM).
-int cluster_capacity(const void* fn, int bits, int gs, int ks) {
+int cluster_capacity(const void* fn, int bits, int gs, int ks, bool swap) {
     constexpr int kDevices = 16;
-    static int cache[kDevices][3][2][9] = {};
-    const int bi = bits == 1 ? 0 : bits == 2 ? 1 : 2, gi = gs == 64 ? 0 : 1;
+    static int cache[kDevices][3][2][2][9] = {};
+    const int bi = bits == 1 ? 0 : bits == 2 ? 1 : 2, gi = gs == 64 ? 0 : 1, si = swap ? 1 : 0;
     int dev = 0;
     cudaGetDevice(&dev);
     const bool cached = dev >= 0 && dev < kDevices;
     if (cached) {
         std::lock_guard<std::mutex> lock(g_mu);
-        if (cache[dev][bi][gi][ks] > 0) return cache[dev][bi][gi][ks];
+        if (cache[dev][bi][gi][si][ks] > 0) return cache[dev][bi][gi][si][ks];
     }
     int n = 0;
     cudaLaunchConfig_t cfg = {};
@@ -74,7 +75,7 @@ int cluster_capacity(const void* fn, int bits, int gs, int ks) {
     if (n <= 0) n = 1;
     if (cached) {
         std::lock_guard<std::mutex> lock(g_mu);
-        cache[dev][bi][gi][ks] = n;
+        cache[dev][bi][gi][si][ks] = n;
     }
     return n;
 }
@@ -84,8 +85,10 @@ struct Choice {
 };
 
 // Rows per CTA and K slices: the fewest waves of the largest per-CTA share (rows x K slice),
-// rows counted at least 48 since fewer leave too few MMA chains to cover their latency.
-Choice choose(const void* probe, int bits, int gs, int N, int K, int force_rows, int force_split) {
+// rows counted at least 48 since fewer leave too few MMA chains to cover their latency. Rows
+// come in multiples of `align` (8, or 16 with weights as the 16-row operand).
+Choice choose(const void* probe, int bits, int gs, int N, int K, int force_rows, int force_split, bool swap) {
+    const int align = swap ? 16 : 8;
     Choice best{0, 0, 0, 0};
     double best_cost = 0;
     for (int ks = 1; ks <= 8; ++ks) {
@@ -93,11 +96,11 @@ Choice choose(const void* probe, int bits, int gs, int N, int K, int force_rows,
         const int kslice = ((K + ks * kStepK - 1) / (ks * kStepK)) * kStepK;
         const int ks_eff = (K + kslice - 1) / kslice;
         if (!force_split && ks_eff != ks) continue;
-        const int cap = cluster_capacity(probe, bits, gs, ks_eff);
+        const int cap = cluster_capacity(probe, bits, gs, ks_eff, swap);
         int rows = force_rows;
         if (!rows) {
-            rows = 8 * ((N + 8 * cap - 1) / (8 * cap));
-            if (rows < 8) rows = 8;
+            rows = align * ((N + align * cap - 1) / (align * cap));
+            if (rows < align) rows = align;
             if (rows > kMaxRows) rows = kMaxRows;
         }
         const int nb = (N + rows - 1) / rows;
@@ -112,17 +115,17 @@ Choice choose(const void* probe, int bits, int gs, int N, int K, int force_rows,
 }
 
 template <int BITS, int GS>
-lowbit_status launch(const GemmProblem& g, int force_rows, int force_split, cudaStream_t stream) {
+lowbit_status launch(const GemmProblem& g, int force_rows, int force_split, bool swap, cudaStream_t stream) {
     using F = Fmt<BITS, GS>;
     const int M = static_cast<int>(g.M), N = static_cast<int>(g.N), K = static_cast<int>(g.K);
-    const void* probe = kernel_for(BITS, GS, 8);
+    const void* probe = kernel_for(BITS, GS, 8, swap);
     if (!probe || !prepare(probe)) return LOWBIT_ERR_CUDA;
-    const Choice ch = choose(probe, BITS, GS, N, K, force_rows, force_split);
-    const void* fn = kernel_for(BITS, GS, ch.rows / 8);
+    const Choice ch = choose(probe, BITS, GS, N, K, force_rows, force_split, swap);
+    const void* fn = kernel_for(BITS, GS, ch.rows / 8, swap);
     if (!fn || !prepare(fn)) return LOWBIT_ERR_CUDA;
     Params p;
     int smem = 0;
-    if (!layout<BITS, GS>(ch.rows, ch.ksplit, &p, &smem)) return LOWBIT_ERR_UNSUPPORTED;
+    if (!layout<BITS, GS>(ch.rows, ch.ksplit, swap, &p, &smem)) return LOWBIT_ERR_UNSUPPORTED;
     p.M = M;
     p.N = N;
     p.K = K;
@@ -136,7 +139,7 @@ lowbit_status launch(const GemmProblem& g, int force_rows, int force_split, cuda
     CUtensorMap mx, mw, ms, mz;
     const uint64_t xdims[3] = {64, static_cast<uint64_t>(M), static_cast<uint64_t>(K) / 64};
     const uint64_t xstr[2] = {static_cast<uint64_t>(K) * 2, 128};
-    const uint32_t xbox[3] = {64, kTokens, kStepK / 64};
+    const uint32_t xbox[3] = {64, static_cast<uint32_t>(swap ? kSwapTokens : kTokens), kStepK / 64};
     bool ok = make_map_3d(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.X, xdims, xstr, xbox, CU_TENSOR_MAP_SWIZZLE_128B);
     ok = ok && make_map_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, g.Wp, uint64_t(K) * BITS / 32, N,
                            uint64_t(K) * BITS / 8, F::kWBoxWords, ch.rows,
@@ -170,6 +173,7 @@ lowbit_status launch(const GemmProblem& g, int force_rows, int force_split, cuda
     cfg.attrs = attrs;
     cfg.numAttrs = na;
     void* args[] = {&mx, &mw, &ms, &mz, &p};
+    if (take_injected_failure(kInjectLaunch)) return LOWBIT_ERR_CUDA;
     return cudaLaunchKernelExC(&cfg, fn, args) == cudaSuccess ? LOWBIT_OK : LOWBIT_ERR_CUDA;
 }
 
@@ -178,17 +182,17 @@ lowbit_status launch(const GemmProblem& g, int force_rows, int force_split, cuda
 
 bool smallm_supported(const GemmProblem& g) { return g.M >= 1 && g.M <= smallm::kTokens; }
 
-lowbit_status smallm_launch(const GemmProblem& g, int rows, int ksplit, cudaStream_t stream) {
-    if (!smallm_supported(g)) return LOWBIT_ERR_UNSUPPORTED;
-    if (rows < 0 || rows > smallm::kMaxRows || rows % 8 != 0 || ksplit < 0 || ksplit > 8)
+lowbit_status smallm_launch(const GemmProblem& g, int rows, int ksplit, bool swap, cudaStream_t stream) {
+    if (!smallm_supported(g) || (swap && g.M > smallm::kSwapTokens)) return LOWBIT_ERR_UNSUPPORTED;
+    if (rows < 0 || rows > smallm::kMaxRows || rows % (swap ? 16 : 8) != 0 || ksplit < 0 || ksplit > 8)
         return LOWBIT_ERR_UNSUPPORTED;
     switch (g.bits * 1000 + g.group_size) {
-        case 1064: return smallm::launch<1, 64>(g, rows, ksplit, stream);
-        case 1128: return smallm::launch<1, 128>(g, rows, ksplit, stream);
-        case 2064: return smallm::launch<2, 64>(g, rows, ksplit, stream);
-        case 2128: return smallm::launch<2, 128>(g, rows, ksplit, stream);
-        case 4064: return smallm::launch<4, 64>(g, rows, ksplit, stream);
-        case 4128: return smallm::launch<4, 128>(g, rows, ksplit, stream);
+        case 1064: return smallm::launch<1, 64>(g, rows, ksplit, swap, stream);
+        case 1128: return smallm::launch<1, 128>(g, rows, ksplit, swap, stream);
+        case 2064: return smallm::launch<2, 64>(g, rows, ksplit, swap, stream);
+        case 2128: return smallm::launch<2, 128>(g, rows, ksplit, swap, stream);
+        case 4064: return smallm::launch<4, 64>(g, rows, ksplit, swap, stream);
+        case 4128: return smallm::launch<4, 128>(g, rows, ksplit, swap, stream);
         default: return LOWBIT_ERR_UNSUPPORTED;
     }
 }

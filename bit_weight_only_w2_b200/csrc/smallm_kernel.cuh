@@ -62,12 +62,14 @@ constexpr int kHalves = 1;
 constexpr int kWarps = kKWarps * kHalves;
 constexpr int kThreads = kWarps * 32;
 constexpr int kStepK = 512;                       // K per ring step
-constexpr int kTokens = 16;
+constexpr int kTokens = 16;                       // tokens per MMA tile, X as the 16-row operand
+constexpr int kSwapTokens = 8;                    // tokens per MMA tile, weights as the 16-row operand
 constexpr int kMaxRows = 128;
 constexpr int kMaxOct = kMaxRows / 8;
-constexpr int kMaxChains = kHalves == 1 ? 12 : 5;  // octet chains interleaved per sub-batch
+constexpr int kMaxChains = kHalves == 1 ? 12 : 5;  // accumulator chains interleaved per sub-batch
 constexpr int kMaxStages = 8;
-constexpr int kXBytes = kTokens * kStepK * 2;     // X slice of one step: 16 KB
+// X slice of one step: [tokens][512] bf16 (16 KB, or 8 KB with weights as the 16-row operand)
+constexpr int x_bytes(bool swap) { return (swap ? kSwapTokens : kTokens) * kStepK * 2; }
 constexpr int kSmemLimit = 227 * 1024;
 constexpr int kBarBytes = 256;
 constexpr uint32_t kBf16One2 = 0x3F803F80u;       // bf16 pair (1, 1)
@@ -91,26 +93,30 @@ struct Params {
     unsigned* status;     // the device status word (bounded waits record timeouts here)
 };
 
-// Shared-memory layout for `rows` weight rows per tile. Every TMA destination starts on a
-// 128-byte boundary (1024 for the swizzled X and code boxes). Returns false if fewer than two
-// ring stages fit.
+// Shared-memory layout for `rows` weight rows per tile (a multiple of 16 when `swap`). Every TMA
+// destination starts on a 128-byte boundary (1024 for the swizzled X and code boxes). Returns
+// false if fewer than two ring stages fit. A tile's MMA units are its octets of rows, or with
+// `swap` its pairs of octets (16 rows, the A operand's height).
 template <int BITS, int GS>
-bool layout(int rows, int ksplit, Params* p, int* smem_bytes) {
+bool layout(int rows, int ksplit, bool swap, Params* p, int* smem_bytes) {
     using F = Fmt<BITS, GS>;
-    const int noct = rows / 8;
+    const int units = swap ? rows / 16 : rows / 8;
+    const uint32_t xb = x_bytes(swap);
     const uint32_t w_bytes = F::kWBoxes * rows * F::kWRow;   // a multiple of 512
     const uint32_t s_raw = F::kGroups * rows * 2;
     const uint32_t s_bytes = (s_raw + 127) / 128 * 128;
-    p->w_off = kXBytes;
+    p->w_off = xb;
     p->s_off = p->w_off + w_bytes;
     p->z_off = p->s_off + s_bytes;
     const uint32_t end = p->z_off + (BITS == 4 ? s_bytes : 0);
     p->stage_bytes = (end + 1023) / 1024 * 1024;
-    p->tx_bytes = kXBytes + w_bytes + s_raw * (BITS == 4 ? 2 : 1);
-    const uint32_t scr = kWarps * 4 * ((noct + kHalves - 1) / kHalves) * 16;   // per warp: (s, s * c) pairs of its rows
-    const uint32_t red = 4 * noct * 512;
-    // receive buffer of the octets this rank finishes: [ksplit][ceil(noct / ksplit)][32 lanes]
-    const uint32_t part = ksplit > 1 ? ksplit * ((noct + ksplit - 1) / ksplit) * 512 : 0;
+    p->tx_bytes = xb + w_bytes + s_raw * (BITS == 4 ? 2 : 1);
+    // per warp, fp32 (s, s * c) of its rows: four float4 per octet (pairs of rows), or eight per
+    // unit with `swap` (rows g and g + 8 of the unit for each g)
+    const uint32_t scr = kWarps * (swap ? 8 : 4) * ((units + kHalves - 1) / kHalves) * 16;
+    const uint32_t red = 4 * units * 512;
+    // receive buffer of the units this rank finishes: [ksplit][ceil(units / ksplit)][32 lanes]
+    const uint32_t part = ksplit > 1 ? ksplit * ((units + ksplit - 1) / ksplit) * 512 : 0;
     const int fixed = static_cast<int>(scr + red + part) + kBarBytes + 1024;
     int stages = (kSmemLimit - fixed) / static_cast<int>(p->stage_bytes);
     if (stages > kMaxStages) stages = kMaxStages;
@@ -176,19 +182,23 @@ __device__ __forceinline__ uint32_t dec_b1(uint32_t v, int c) {       // +-1 by 
     return xor_andnot(0x3F803F80u, v << (15 - c), 0x80008000u);
 }
 
-template <int BITS, int GS, int NOCT>
+template <int BITS, int GS, int NOCT, bool SWAP>
 __global__ void __launch_bounds__(kThreads, 1)
     lowbit_smallm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w,
                          const __grid_constant__ CUtensorMap map_s, const __grid_constant__ CUtensorMap map_z,
                          const Params p) {
     using F = Fmt<BITS, GS>;
+    static_assert(!SWAP || NOCT % 2 == 0, "weights as the 16-row operand take rows in pairs of octets");
     constexpr int R = 8 * NOCT;                       // weight rows per tile
     constexpr int HALF = R / 2;                       // (s, s * c) pairs per group
-    constexpr int NH = (NOCT + kHalves - 1) / kHalves; // octets per warp (its half of the tile)
-    constexpr int HP = 4 * NH;                        // (s, s * c) pairs of a half's rows
+    constexpr int NUT = SWAP ? NOCT / 2 : NOCT;       // MMA units per tile: octets, or 16-row pairs of octets
+    constexpr int NH = (NUT + kHalves - 1) / kHalves; // units per warp (its half of the tile)
+    constexpr int HP = (SWAP ? 8 : 4) * NH;           // scale-table entries of a warp
     constexpr int NB = (NH + kMaxChains - 1) / kMaxChains;
-    constexpr int B = (NH + NB - 1) / NB;             // octets per sub-batch
+    constexpr int B = (NH + NB - 1) / NB;             // units per sub-batch
     constexpr int WPS = BITS == 4 ? 2 : BITS == 2 ? 1 : 2;   // code words per lane per octet per step
+    constexpr int OPU = SWAP ? 2 : 1;                 // octets per unit
+    constexpr uint32_t kAtomBytes = (SWAP ? kSwapTokens : kTokens) * 128;   // one 64-wide k-atom of X
     if (threadIdx.x == 0) {
         tma_prefetch_desc(&map_x);
         tma_prefetch_desc(&map_w);
@@ -265,13 +275,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     const int w = warp & (kKWarps - 1);      // this warp's 64-wide K chunk of every step
-    const int ob0 = (warp / kKWarps) * NH;   // first octet of this warp's half of the tile
-    const int nh = (NOCT % kHalves == 0) ? NH : min(NH, NOCT - ob0);   // octets it owns
-    const int g = lane >> 2;                 // B column (weight row in the octet) / C row
+    const int ob0 = (warp / kKWarps) * NH;   // first unit of this warp's half of the tile
+    const int nh = (NUT % kHalves == 0) ? NH : min(NH, NUT - ob0);   // units it owns
+    const int g = lane >> 2;                 // fragment row group: weight row in the octet (B / A rows)
     const int q = lane & 3;
     const int gi = (w * 64) / GS;            // this warp's group within a step
-    const int tok = lane & 15;               // ldmatrix row (token) supplied by this lane
-    const uint32_t xoff = static_cast<uint32_t>(w * 2048 + tok * 128);
+    // X fragments: with X as the 16-row A operand, lane supplies token lane & 15 of k half lane >> 4;
+    // with weights as A, X is the n8 B operand and lane supplies token lane & 7 of 16-byte chunk
+    // lane >> 3 (plus 4 for the second pair of K steps).
+    const int tok = SWAP ? (lane & 7) : (lane & 15);
+    const uint32_t xoff = static_cast<uint32_t>(w * kAtomBytes + tok * 128);
     const int xhalf = lane >> 4;
     // This lane's code bytes in row g of octet 0 of a step (swizzled as the TMA wrote them; the
     // swizzle depends on the row only through g, so octet o is at a fixed offset from it). 2- and
@@ -304,59 +317,101 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (ok) {
                 const uint8_t* st = ring + s * p.stage_bytes;
                 const uint32_t st_u = smem_u32(st);
-                // this warp's group: fp32 (s, s * c) for every pair of rows of its octets
+                // this warp's group: fp32 (s, s * c) of every row of its units
                 {
-                    const __half2* sp = reinterpret_cast<const __half2*>(st + p.s_off) + gi * HALF + 4 * ob0;
-                    const __half2* zp = reinterpret_cast<const __half2*>(st + p.z_off) + gi * HALF + 4 * ob0;
+                    const __half* sh = reinterpret_cast<const __half*>(st + p.s_off) + gi * R;
+                    const __half* zh = reinterpret_cast<const __half*>(st + p.z_off) + gi * R;
+                    auto sc_of = [&](int r, float& sf, float& cf) {
+                        sf = __half2float(sh[r]);
+                        cf = BITS == 4 ? sf * (128.f + __half2float(zh[r])) : BITS == 2 ? 129.f * sf : 0.f;
+                    };
+                    if constexpr (SWAP) {
+                        // entry 8u + g: rows 16u + g and 16u + g + 8 of the warp's units
 #pragma unroll
-                    for (int i0 = 0; i0 < HP; i0 += 32) {
-                        const int i = i0 + lane;
-                        if (i < 4 * nh) {
-                            const float2 sf = __half22float2(sp[i]);
-                            float c0 = 0.f, c1 = 0.f;
-                            if (BITS == 4) {
-                                const float2 zf = __half22float2(zp[i]);
-                                c0 = sf.x * (128.f + zf.x);
-                                c1 = sf.y * (128.f + zf.y);
-                            } else if (BITS == 2) {
-                                c0 = 129.f * sf.x;
-                                c1 = 129.f * sf.y;
+                        for (int i0 = 0; i0 < HP; i0 += 32) {
+                            const int i = i0 + lane;
+                            if (i < 8 * nh) {
+                                const int r = 16 * (ob0 + (i >> 3)) + (i & 7);
+                                float s0, c0, s1, c1;
+                                sc_of(r, s0, c0);
+                                sc_of(r + 8, s1, c1);
+                                scr[i] = make_float4(s0, s1, c0, c1);
                             }
-                            scr[i] = make_float4(sf.x, sf.y, c0, c1);
+                        }
+                    } else {
+                        const __half2* sp = reinterpret_cast<const __half2*>(sh) + 4 * ob0;
+                        const __half2* zp = reinterpret_cast<const __half2*>(zh) + 4 * ob0;
+#pragma unroll
+                        for (int i0 = 0; i0 < HP; i0 += 32) {
+                            const int i = i0 + lane;
+                            if (i < 4 * nh) {
+                                const float2 sf = __half22float2(sp[i]);
+                                float c0 = 0.f, c1 = 0.f;
+                                if (BITS == 4) {
+                                    const float2 zf = __half22float2(zp[i]);
+                                    c0 = sf.x * (128.f + zf.x);
+                                    c1 = sf.y * (128.f + zf.y);
+                                } else if (BITS == 2) {
+                                    c0 = 129.f * sf.x;
+                                    c1 = 129.f * sf.y;
+                                }
+                                scr[i] = make_float4(sf.x, sf.y, c0, c1);
+                            }
                         }
                     }
                     // (read back by the other lanes only after the first sub-batch's MMAs)
                 }
-                // X fragments of this warp's four 16-wide K steps (128-byte swizzled rows)
+                // X fragments of this warp's four 16-wide K steps (128-byte swizzled rows):
+                // a[j] = the A operand of step j, or with SWAP a[p] = the B operands of steps 2p, 2p + 1
                 uint32_t a[4][4];
+                if constexpr (SWAP) {
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int chunk = (j << 1) | xhalf;
-                    ldmatrix_x4(st_u + xoff + static_cast<uint32_t>((chunk ^ (tok & 7)) << 4), a[j]);
+                    for (int pp = 0; pp < 2; ++pp) {
+                        const int chunk = 4 * pp + (lane >> 3);
+                        ldmatrix_x4(st_u + xoff + static_cast<uint32_t>((chunk ^ tok) << 4), a[pp]);
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int chunk = (j << 1) | xhalf;
+                        ldmatrix_x4(st_u + xoff + static_cast<uint32_t>((chunk ^ (tok & 7)) << 4), a[j]);
+                    }
                 }
-                float tsx[4] = {0.f, 0.f, 0.f, 0.f};   // group sums of X: tokens g (0), g + 8 (2)
+                // group sums of X: tokens g (0) and g + 8 (2), or with SWAP tokens 2q (0) and 2q + 1 (1)
+                float tsx[4] = {0.f, 0.f, 0.f, 0.f};
                 if (BITS != 1) {
-                    mma_bf16_z(tsx, a[0], kBf16One2, kBf16One2);
+                    if constexpr (SWAP) {
+                        const uint32_t ones[4] = {kBf16One2, kBf16One2, kBf16One2, kBf16One2};
+                        mma_bf16_z(tsx, ones, a[0][0], a[0][1]);
+                        mma_bf16(tsx, ones, a[0][2], a[0][3]);
+                        mma_bf16(tsx, ones, a[1][0], a[1][1]);
+                        mma_bf16(tsx, ones, a[1][2], a[1][3]);
+                    } else {
+                        mma_bf16_z(tsx, a[0], kBf16One2, kBf16One2);
 #pragma unroll
-                    for (int j = 1; j < 4; ++j) mma_bf16(tsx, a[j], kBf16One2, kBf16One2);
+                        for (int j = 1; j < 4; ++j) mma_bf16(tsx, a[j], kBf16One2, kBf16One2);
+                    }
                 }
                 const uint8_t* wst = st + p.w_off;
 #pragma unroll
                 for (int ob = 0; ob < NH; ob += B) {
-                    // codes of the sub-batch's octets for this warp's 64 K
-                    uint32_t wd[B][WPS];
+                    // codes of the sub-batch's units for this warp's 64 K
+                    uint32_t wd[B][OPU][WPS];
 #pragma unroll
                     for (int u = 0; u < B; ++u) {
                         if (ob + u < nh) {
-                            const uint8_t* rp = wst + (ob0 + ob + u) * kOctStride;
-                            if (BITS == 4) {
-                                wd[u][0] = *reinterpret_cast<const uint32_t*>(rp + wb0);
-                                wd[u][1] = *reinterpret_cast<const uint32_t*>(rp + wb1);
-                            } else if (BITS == 2) {
-                                wd[u][0] = *reinterpret_cast<const uint32_t*>(rp + wb0);
-                            } else {
-                                const uint2 v = *reinterpret_cast<const uint2*>(rp + wb0);
-                                wd[u][0] = v.x; wd[u][1] = v.y;
+#pragma unroll
+                            for (int h = 0; h < OPU; ++h) {
+                                const uint8_t* rp = wst + (OPU * (ob0 + ob + u) + h) * kOctStride;
+                                if (BITS == 4) {
+                                    wd[u][h][0] = *reinterpret_cast<const uint32_t*>(rp + wb0);
+                                    wd[u][h][1] = *reinterpret_cast<const uint32_t*>(rp + wb1);
+                                } else if (BITS == 2) {
+                                    wd[u][h][0] = *reinterpret_cast<const uint32_t*>(rp + wb0);
+                                } else {
+                                    const uint2 v = *reinterpret_cast<const uint2*>(rp + wb0);
+                                    wd[u][h][0] = v.x; wd[u][h][1] = v.y;
+                                }
                             }
                         }
                     }
@@ -366,38 +421,66 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int u = 0; u < B; ++u) {
                             if (ob + u < nh) {
-                                uint32_t b0, b1;
-                                if (BITS == 4) {           // block j / 2, pairs 2(j % 2) and + 1
-                                    b0 = dec_u4(wd[u][j >> 1], 2 * (j & 1));
-                                    b1 = dec_u4(wd[u][j >> 1], 2 * (j & 1) + 1);
-                                } else if (BITS == 2) {    // the chunk's block, pairs 2j and 2j + 1
-                                    b0 = dec_t2(wd[u][0], 2 * j);
-                                    b1 = dec_t2(wd[u][0], 2 * j + 1);
-                                } else {
-                                    const int pc = (j & 1) * 8 + q;
-                                    b0 = dec_b1(wd[u][j >> 1], pc);
-                                    b1 = dec_b1(wd[u][j >> 1], pc + 4);
+                                // (b0, b1): row g's codes for k = 2q, 2q + 1 and 2q + 8, 2q + 9 of step j
+                                uint32_t b0[OPU], b1[OPU];
+#pragma unroll
+                                for (int h = 0; h < OPU; ++h) {
+                                    if (BITS == 4) {           // block j / 2, pairs 2(j % 2) and + 1
+                                        b0[h] = dec_u4(wd[u][h][j >> 1], 2 * (j & 1));
+                                        b1[h] = dec_u4(wd[u][h][j >> 1], 2 * (j & 1) + 1);
+                                    } else if (BITS == 2) {    // the chunk's block, pairs 2j and 2j + 1
+                                        b0[h] = dec_t2(wd[u][h][0], 2 * j);
+                                        b1[h] = dec_t2(wd[u][h][0], 2 * j + 1);
+                                    } else {
+                                        const int pc = (j & 1) * 8 + q;
+                                        b0[h] = dec_b1(wd[u][h][j >> 1], pc);
+                                        b1[h] = dec_b1(wd[u][h][j >> 1], pc + 4);
+                                    }
                                 }
-                                if (j == 0) mma_bf16_z(T[u], a[0], b0, b1);
-                                else mma_bf16(T[u], a[j], b0, b1);
+                                if constexpr (SWAP) {
+                                    // A = rows g (octet 2u) and g + 8 (octet 2u + 1) of the unit
+                                    const uint32_t aw[4] = {b0[0], b0[OPU - 1], b1[0], b1[OPU - 1]};
+                                    const uint32_t x0 = a[j >> 1][2 * (j & 1)], x1 = a[j >> 1][2 * (j & 1) + 1];
+                                    if (j == 0) mma_bf16_z(T[u], aw, x0, x1);
+                                    else mma_bf16(T[u], aw, x0, x1);
+                                } else {
+                                    if (j == 0) mma_bf16_z(T[u], a[0], b0[0], b1[0]);
+                                    else mma_bf16(T[u], a[j], b0[0], b1[0]);
+                                }
                             }
                         }
                     }
-                    if (ob == 0) __syncwarp();   // the scale pairs above are written
+                    if (ob == 0) __syncwarp();   // the scale entries above are written
 #pragma unroll
                     for (int u = 0; u < B; ++u) {
                         if (ob + u < nh) {
-                            const float4 sc = scr[4 * (ob + u) + q];
                             float* d = acc[ob + u];
-                            d[0] = fmaf(sc.x, T[u][0], d[0]);
-                            d[1] = fmaf(sc.y, T[u][1], d[1]);
-                            d[2] = fmaf(sc.x, T[u][2], d[2]);
-                            d[3] = fmaf(sc.y, T[u][3], d[3]);
-                            if (BITS != 1) {
-                                d[0] = fmaf(-sc.z, tsx[0], d[0]);
-                                d[1] = fmaf(-sc.w, tsx[0], d[1]);
-                                d[2] = fmaf(-sc.z, tsx[2], d[2]);
-                                d[3] = fmaf(-sc.w, tsx[2], d[3]);
+                            if constexpr (SWAP) {
+                                // d: (row g, token 2q), (row g, 2q + 1), (row g + 8, 2q), (row g + 8, 2q + 1)
+                                const float4 sc = scr[8 * (ob + u) + g];
+                                d[0] = fmaf(sc.x, T[u][0], d[0]);
+                                d[1] = fmaf(sc.x, T[u][1], d[1]);
+                                d[2] = fmaf(sc.y, T[u][2], d[2]);
+                                d[3] = fmaf(sc.y, T[u][3], d[3]);
+                                if (BITS != 1) {
+                                    d[0] = fmaf(-sc.z, tsx[0], d[0]);
+                                    d[1] = fmaf(-sc.z, tsx[1], d[1]);
+                                    d[2] = fmaf(-sc.w, tsx[0], d[2]);
+                                    d[3] = fmaf(-sc.w, tsx[1], d[3]);
+                                }
+                            } else {
+                                // d: (token g, row 2q), (g, 2q + 1), (g + 8, 2q), (g + 8, 2q + 1)
+                                const float4 sc = scr[4 * (ob + u) + q];
+                                d[0] = fmaf(sc.x, T[u][0], d[0]);
+                                d[1] = fmaf(sc.y, T[u][1], d[1]);
+                                d[2] = fmaf(sc.x, T[u][2], d[2]);
+                                d[3] = fmaf(sc.y, T[u][3], d[3]);
+                                if (BITS != 1) {
+                                    d[0] = fmaf(-sc.z, tsx[0], d[0]);
+                                    d[1] = fmaf(-sc.w, tsx[0], d[1]);
+                                    d[2] = fmaf(-sc.z, tsx[2], d[2]);
+                                    d[3] = fmaf(-sc.w, tsx[2], d[3]);
+                                }
                             }
                         }
                     }
@@ -419,13 +502,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
 
-        // ---- tile end: every octet's eight K-chunk partials (one per warp of its half) are added
+        // ---- tile end: every unit's eight K-chunk partials (one per warp of its half) are added
         // in a fixed order. On a CTA's only tile the drained ring holds all eight: one exchange,
         // ((((c0 + c1) + c2) + ...) + c7). Otherwise the ring already holds the next tile's steps
         // and `red` takes two rounds: (c + (c + 4)) for chunks c < 4, then ((0 + 1) + 2) + 3.
         grid_dependency_wait();   // Y may still be read by the kernel this one overlaps
         const bool one_round =
-            my_tiles == 1 && static_cast<uint32_t>(S) * p.stage_bytes >= kKWarps * NOCT * 512u;
+            my_tiles == 1 && static_cast<uint32_t>(S) * p.stage_bytes >= kKWarps * NUT * 512u;
         float4* rbuf = one_round ? reinterpret_cast<float4*>(ring) : red;
         const int nslot = one_round ? kKWarps : 4;
         cta_bar();                // the ring is drained / the previous tile's readers of `red` are done
@@ -434,7 +517,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int o = 0; o < NH; ++o)
                 if (o < nh)
-                    rbuf[(slot * NOCT + ob0 + o) * 32 + lane] = make_float4(acc[o][0], acc[o][1], acc[o][2], acc[o][3]);
+                    rbuf[(slot * NUT + ob0 + o) * 32 + lane] = make_float4(acc[o][0], acc[o][1], acc[o][2], acc[o][3]);
         }
         cta_bar();
         if (!one_round) {
@@ -442,7 +525,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int o = 0; o < NH; ++o) {
                     if (o < nh) {
-                        const float4 v = red[(w * NOCT + ob0 + o) * 32 + lane];
+                        const float4 v = red[(w * NUT + ob0 + o) * 32 + lane];
                         acc[o][0] += v.x;
                         acc[o][1] += v.y;
                         acc[o][2] += v.z;
@@ -455,7 +538,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int o = 0; o < NH; ++o)
                     if (o < nh)
-                        red[(w * NOCT + ob0 + o) * 32 + lane] = make_float4(acc[o][0], acc[o][1], acc[o][2], acc[o][3]);
+                        red[(w * NUT + ob0 + o) * 32 + lane] = make_float4(acc[o][0], acc[o][1], acc[o][2], acc[o][3]);
             }
             cta_bar();
         }
@@ -464,14 +547,28 @@ __global__ void __launch_bounds__(kThreads, 1)
 
         const int n0 = t * R;
         auto store = [&](int o, float4 v) {
-            const int n = n0 + 8 * o + 2 * q;
-            if (n < p.N) {
-                if (g < p.M)
-                    *reinterpret_cast<__nv_bfloat162*>(p.Y + static_cast<size_t>(g) * p.N + n) =
-                        __floats2bfloat162_rn(v.x, v.y);
-                if (g + 8 < p.M)
-                    *reinterpret_cast<__nv_bfloat162*>(p.Y + static_cast<size_t>(g + 8) * p.N + n) =
-                        __floats2bfloat162_rn(v.z, v.w);
+            if constexpr (SWAP) {
+                // rows n and n + 8 of unit o, tokens 2q and 2q + 1
+                const int n = n0 + 16 * o + g;
+                const int t0 = 2 * q;
+                if (dcheck(o < NUT && n >= 0, p.status)) {
+                    const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int ne = n + (e >> 1) * 8, te = t0 + (e & 1);
+                        if (ne < p.N && te < p.M) p.Y[static_cast<size_t>(te) * p.N + ne] = __float2bfloat16_rn(vv[e]);
+                    }
+                }
+            } else {
+                const int n = n0 + 8 * o + 2 * q;
+                if (n < p.N && dcheck(n >= 0 && n + 1 < p.N && o < NUT, p.status)) {
+                    if (g < p.M)
+                        *reinterpret_cast<__nv_bfloat162*>(p.Y + static_cast<size_t>(g) * p.N + n) =
+                            __floats2bfloat162_rn(v.x, v.y);
+                    if (g + 8 < p.M)
+                        *reinterpret_cast<__nv_bfloat162*>(p.Y + static_cast<size_t>(g + 8) * p.N + n) =
+                            __floats2bfloat162_rn(v.z, v.w);
+                }
             }
         };
         auto tile_sum = [&](int o) {
@@ -479,7 +576,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int r = 1; r < kKWarps; ++r) {
                 if (r >= nslot) break;
-                const float4 u = rbuf[(r * NOCT + o) * 32 + lane];
+                const float4 u = rbuf[(r * NUT + o) * 32 + lane];
                 v.x += u.x;
                 v.y += u.y;
                 v.z += u.z;
@@ -488,19 +585,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             return v;
         };
         if (ks == 1) {
-            for (int o = warp; o < NOCT; o += kWarps) store(o, tile_sum(o));
+            for (int o = warp; o < NUT; o += kWarps) store(o, tile_sum(o));
         } else {
-            // Octet o is finished by rank o % ks: every rank stores its tile sum of o straight into
+            // Unit o is finished by rank o % ks: every rank stores its tile sum of o straight into
             // that rank's receive buffer (slot [own rank][o / ks]); after a cluster barrier the
             // finishing rank adds the slots in rank order; a second barrier keeps the buffers
             // (and every CTA) alive until all ranks have read them.
-            const int per = (NOCT + ks - 1) / ks;
-            for (int o = warp; o < NOCT; o += kWarps) {
+            const int per = (NUT + ks - 1) / ks;
+            for (int o = warp; o < NUT; o += kWarps) {
                 const uint32_t slot = smem_u32(part + ((rank * per + o / ks) * 32 + lane));
                 st_shared_cluster_v4(map_shared_rank(slot, o % ks), tile_sum(o));
             }
             cluster_sync_all();
-            for (int o = warp; o < NOCT; o += kWarps) {
+            for (int o = warp; o < NUT; o += kWarps) {
                 if (o % ks != rank) continue;
                 const int li = o / ks;
                 float4 sum = part[li * 32 + lane];
@@ -527,26 +624,40 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-// Kernel entry for (BITS, GS) and `noct` octets per tile (1..16), or nullptr. One definition
-// per code width lives in its own translation unit so the instantiations build in parallel.
-const void* kernel_b1(int group_size, int noct);
-const void* kernel_b2(int group_size, int noct);
-const void* kernel_b4(int group_size, int noct);
+// Kernel entry for (BITS, GS), `noct` octets per tile (1..16) and the orientation (`swap`:
+// weights as the 16-row operand, even `noct` only), or nullptr. One definition per code width
+// lives in its own translation unit so the instantiations build in parallel.
+const void* kernel_b1(int group_size, int noct, bool swap);
+const void* kernel_b2(int group_size, int noct, bool swap);
+const void* kernel_b4(int group_size, int noct, bool swap);
 
 }  // namespace smallm
 }  // namespace lowbit
 
-// Defines kernel_b<BITS>: a table of the sixteen octet counts for both group sizes.
+// Defines kernel_b<BITS>: tables of the sixteen octet counts (and the eight even ones with weights
+// as the 16-row operand) for both group sizes.
 #define LOWBIT_SMALLM_TABLE(BITS)                                                                     \
     namespace lowbit {                                                                                \
     namespace smallm {                                                                                \
     template <int GS, int... Ns>                                                                      \
     static const void* pick_##BITS(int noct, std::integer_sequence<int, Ns...>) {                     \
         static const void* const table[] = {                                                          \
-            reinterpret_cast<const void*>(&lowbit_smallm_kernel<BITS, GS, Ns + 1>)...};               \
+            reinterpret_cast<const void*>(&lowbit_smallm_kernel<BITS, GS, Ns + 1, false>)...};        \
         return (noct >= 1 && noct <= static_cast<int>(sizeof...(Ns))) ? table[noct - 1] : nullptr;    \
     }                                                                                                 \
-    const void* kernel_b##BITS(int group_size, int noct) {                                            \
+    template <int GS, int... Ns>                                                                      \
+    static const void* pick_swap_##BITS(int noct, std::integer_sequence<int, Ns...>) {                \
+        static const void* const table[] = {                                                          \
+            reinterpret_cast<const void*>(&lowbit_smallm_kernel<BITS, GS, 2 * (Ns + 1), true>)...};   \
+        return (noct >= 2 && noct % 2 == 0 && noct / 2 <= static_cast<int>(sizeof...(Ns)))           \
+                   ? table[noct / 2 - 1] : nullptr;                                                   \
+    }                                                                                                 \
+    const void* kernel_b##BITS(int group_size, int noct, bool swap) {                                 \
+        if (swap) {                                                                                   \
+            if (group_size == 64) return pick_swap_##BITS<64>(noct, std::make_integer_sequence<int, kMaxOct / 2>{}); \
+            if (group_size == 128) return pick_swap_##BITS<128>(noct, std::make_integer_sequence<int, kMaxOct / 2>{}); \
+            return nullptr;                                                                           \
+        }                                                                                             \
         if (group_size == 64) return pick_##BITS<64>(noct, std::make_integer_sequence<int, kMaxOct>{}); \
         if (group_size == 128) return pick_##BITS<128>(noct, std::make_integer_sequence<int, kMaxOct>{}); \
         return nullptr;                                                                               \

@@ -37,10 +37,13 @@
  * Scale / zero layout: fp16, group-major [K/group_size][N]: s(n, k) = scales[(k/g)*N + n].
  * X: bf16 row-major [M][K]. Y: bf16 row-major [M][N].
  *
- * Arithmetic: X is copied to fp16 in the caller's workspace (exactly: each row is first scaled
- * by a power of two that keeps it inside fp16's range, and the result is scaled back), weights
- * are decoded to fp16 (binary / ternary exactly, uint4 with one rounding), products are summed
- * in fp32 on the tensor cores and Y is rounded to bf16 once.
+ * Arithmetic (M > 16): X is copied to fp16 in the caller's workspace (exactly: each row is first
+ * scaled by a power of two that keeps it inside fp16's range, and the result is scaled back);
+ * binary and ternary weights decode to exactly +-s or 0 in fp16; a uint4 weight (q - z) * s is
+ * computed in fp32 (error below 2^-24 relative) and rounded once to fp16; products are summed in
+ * fp32 on the tensor cores and Y is rounded to bf16 once. M <= 16: codes decode exactly without
+ * their scale, X is used as stored (bf16), group sums are formed in fp32 and scaled there (see
+ * lowbit_gemm_ex, tile_tokens = 1).
  *
  * Ownership: the caller owns every buffer (device memory unless stated), including the GEMM
  * workspace (see lowbit_gemm_workspace_size). The library allocates nothing; it holds a few
@@ -67,7 +70,9 @@ typedef enum lowbit_status {
     LOWBIT_ERR_BAD_CODE = 5,           /* pack: a code outside its format; unpack: field 3       */
     LOWBIT_ERR_TIMEOUT = 6,            /* a bounded wait inside a kernel gave up (device status) */
     LOWBIT_ERR_CUDA = 7,               /* a CUDA runtime / driver call failed                    */
-    LOWBIT_ERR_WORKSPACE = 8           /* workspace NULL, misaligned or smaller than required    */
+    LOWBIT_ERR_WORKSPACE = 8,          /* workspace NULL, misaligned or smaller than required    */
+    LOWBIT_ERR_DEVICE_CHECK = 9        /* a device-side index check failed (debug builds only;   */
+                                       /* see lowbit_debug_checks_enabled)                       */
 } lowbit_status;
 
 /* Human-readable name of a status. Never NULL. */
@@ -153,16 +158,32 @@ typedef struct lowbit_gemm_desc {
 
 /* Run `count` GEMMs (host array of descriptors) in order on `stream`, as if lowbit_gemm were
  * called for each in turn with the same workspace: a descriptor may read an earlier one's Y.
+ * This is the unit of one denoise step of the transformer: its 25 MMDiT blocks, 5 double-stream
+ * and 20 single-stream (bonsai-image-binary-4B-gemlite-1bit model card, model overview /
+ * specifications), each run their Q/K/V, output and MLP linears in order.
  * The workspace must hold the largest lowbit_gemm_workspace_size(M, K) of the descriptors.
  * All descriptors are validated first; on any invalid one nothing is launched and its error
  * is returned. Consecutive launches overlap their prologues with the previous kernel's tail
- * (programmatic dependent launch); results are the same as separate calls. */
+ * (programmatic dependent launch); results are the same as separate calls. A linear with more
+ * than 16 tokens that reads the same X as the previous such linear (same pointer, M and K),
+ * with no output written since then overlapping that X, reuses the fp16 copy of X already in
+ * the workspace instead of converting it again (separate Q, K and V projections of one input
+ * convert it once). A failure while launching returns at once; the linears before it have
+ * been queued and will run. */
 lowbit_status lowbit_gemm_batch(const lowbit_gemm_desc* descs, int count, void* workspace,
                                 size_t workspace_bytes, void* stream);
 
 /* Read the current device's sticky status word, written by kernels whose bounded waits gave
- * up (LOWBIT_ERR_TIMEOUT), and clear it when `clear` != 0. Synchronises the device. */
+ * up (LOWBIT_ERR_TIMEOUT) or, in debug builds, whose index checks failed
+ * (LOWBIT_ERR_DEVICE_CHECK), and clear it when `clear` != 0. Synchronises the whole device. */
 lowbit_status lowbit_device_status(int clear);
+
+/* Debug: the same status word read in stream order -- the read and the clearing of the word are
+ * queued on `stream` and only that stream is waited for, so other streams keep running. The
+ * word is per device: it also reports kernels of other streams that finished before the read.
+ * Returns LOWBIT_OK, LOWBIT_ERR_TIMEOUT or LOWBIT_ERR_DEVICE_CHECK (then clears the word), or
+ * LOWBIT_ERR_CUDA if the copy could not be made. */
+lowbit_status lowbit_last_device_status(void* stream);
 
 /* Size of the static device scratch used by lowbit_gemm_noalloc: 32 MiB. */
 #define LOWBIT_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
@@ -195,6 +216,29 @@ lowbit_status lowbit_gemm_noalloc(int64_t M, int64_t N, int64_t K, int bits, int
  * the device status word and the kernel returns normally, so the context stays usable; read it
  * with lowbit_device_status. Asynchronous. */
 lowbit_status lowbit_selftest_bounded_wait(long long limit_cycles, void* stream);
+
+/* Failure injection, for tests of the error paths: `what` = 1 makes the next tensor-map encode
+ * fail, 2 the next kernel launch (either of the GEMM's two launches counts), 3 both; 0 cancels
+ * what is still pending. Each injected failure fires once, in any thread of the process, at the
+ * point where the real failure would be detected: the call then returns LOWBIT_ERR_CUDA before
+ * launching the affected kernel, exactly as it does when the driver reports the failure. No
+ * kernel is launched differently and no GPU fault is involved. Returns LOWBIT_ERR_INVALID_ARG
+ * for other values. The paper has no counterpart; this is test support. */
+lowbit_status lowbit_test_fail_next(int what);
+
+/* 1 if this library was built with device-side index checks (LOWBIT_DEBUG_CHECKS, shipped as
+ * liblowbit_debug.so), else 0. In such a build every global store of Y, every load of a row
+ * factor and every tensor-memory store of decoded weights first checks its index against the
+ * problem's bounds; a failed check records LOWBIT_ERR_DEVICE_CHECK in the device status word
+ * and skips the access instead of trapping, so the context stays usable. */
+int lowbit_debug_checks_enabled(void);
+
+/* Diagnostic for the debug build's index checks: launches one thread whose store index is one
+ * past its one-element target. The store is made only when the index is in range, so nothing is
+ * written out of bounds in any build; a debug build also records LOWBIT_ERR_DEVICE_CHECK in the
+ * device status word. Returns LOWBIT_ERR_UNSUPPORTED (launching nothing) in release builds.
+ * Asynchronous. */
+lowbit_status lowbit_selftest_index_check(void* stream);
 
 #ifdef __cplusplus
 }

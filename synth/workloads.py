@@ -151,6 +151,20 @@ def text_encoder_mlp_layers(tokens: int, layers: int = 4) -> List[LinearSpec]:
     return out
 
 
+def klein_linears_small_m(tokens: int, bits: int) -> List[LinearSpec]:
+    """The six distinct linear shapes of a denoise step (double-stream QKV d -> 3d, out d -> d,
+    MLP-up d -> 3d, MLP-down 3d -> d; single-stream QKV+MLP-in d -> 6d, out 4d -> d) at a handful
+    of tokens, as a decode-style or text-stream call would run them: ternary (P(0) = 0.4) or
+    binary codes, group 128."""
+    fmt = dict(bits=bits, group_size=128, p0=0.4, scale_lo=0.005, scale_hi=0.02)
+    name = "ternary" if bits == 2 else "binary"
+    out: List[LinearSpec] = []
+    for j, (lname, k, n) in enumerate((("qkv", D, 3 * D), ("out", D, D), ("mlp_up", D, 3 * D), ("mlp_down", 3 * D, D),
+                                       ("qkv_mlp_in", D, 6 * D), ("single_out", 4 * D, D))):
+        out.append(LinearSpec(f"{lname}_m{tokens}_{name}", tokens, k, n, seed=tokens, stream_base=10 * (j + 1), **fmt))
+    return out
+
+
 WORKLOADS = {
     # tiny ternary, uniform codes, group 64
     "tiny_ternary_g64": [LinearSpec("tiny", 64, 256, 512, bits=2, group_size=64, p0=1.0 / 3.0)],
@@ -181,4 +195,7 @@ WORKLOADS = {
     # four text-encoder MLP layers (gate, up, down) at 512 and at 16 tokens
     "te_mlp4_m512_uint4_g64": text_encoder_mlp_layers(512),
     "te_mlp4_m16_uint4_g64": text_encoder_mlp_layers(16),
+    # the transformer's ternary and binary linear shapes at 1, 4 and 16 tokens (HBM-bound)
+    **{f"klein_linears_m{m}_{'ternary' if b == 2 else 'binary'}_g128": klein_linears_small_m(m, b)
+       for b in (2, 1) for m in (1, 4, 16)},
 }

@@ -129,3 +129,87 @@ def test_binding_workspace_size_matches_library():
     import bit_weight_only_w2_b200 as lb
     for M, K in [(1, 64), (16, 2560), (512, 9728), (4608, 12288), (7, 192), (0, 64), (3, 128)]:
         assert lb._workspace_size_fast(M, K) == lb.workspace_size(M, K), (M, K)
+
+
+def test_status_strings_cover_the_enum(lib):
+    for code, name in lb.STATUS.items():
+        assert lib.lowbit_status_string(code) == name.encode()
+
+
+def test_fail_next_validates_its_argument(lib):
+    assert lib.lowbit_test_fail_next(-1) == 1
+    assert lib.lowbit_test_fail_next(4) == 1
+    assert lib.lowbit_test_fail_next(0) == 0      # cancel: nothing pending afterwards
+
+
+def test_debug_build_exports_the_same_abi():
+    """liblowbit_debug.so (device-side index checks) exports every declared entry point and says
+    it is the checked build; the release build says it is not and launches no self-test."""
+    dbg = lb.load_debug()
+    for name in declared_functions():
+        assert hasattr(dbg, name), f"{name} missing from the debug build"
+    assert dbg.lowbit_debug_checks_enabled() == 1
+    rel = lb.load()
+    assert rel.lowbit_debug_checks_enabled() == 0
+    assert rel.lowbit_selftest_index_check(None) == 3     # LOWBIT_ERR_UNSUPPORTED, before any CUDA call
+
+
+# ---- the Python binding checks shapes and devices before calling the library (CPU tensors: the
+# shape checks come first, so a mismatch is reported before the CUDA-device check)
+def _cpu_args(M=16, N=128, K=256, bits=2, g=128):
+    import torch
+    x = torch.zeros((M, K), dtype=torch.bfloat16)
+    packed = torch.zeros((N, K * bits // 32), dtype=torch.int32)
+    s = torch.zeros((K // g, N), dtype=torch.float16)
+    z = torch.zeros((K // g, N), dtype=torch.float16) if bits == 4 else None
+    return x, packed, s, z
+
+
+@pytest.mark.parametrize("bad,match", [
+    ("packed_rows", "packed: expected shape"),
+    ("packed_cols", "packed: expected shape"),
+    ("scales_transposed", "scales: expected shape"),
+    ("zeros_shape", "zeros: expected the scales' shape"),
+    ("out_shape", "out: expected shape"),
+    ("x_1d", "x: expected a contiguous 2-D"),
+    ("packed_dtype", "packed: expected a contiguous"),
+    ("x_noncontig", "x: expected a contiguous"),
+])
+def test_binding_rejects_mismatched_tensors(bad, match):
+    import torch
+    bits = 4 if bad == "zeros_shape" else 2
+    g = 64 if bits == 4 else 128
+    x, packed, s, z = _cpu_args(bits=bits, g=g)
+    out = None
+    if bad == "packed_rows":
+        packed = torch.zeros((120, packed.shape[1]), dtype=torch.int32)
+    elif bad == "packed_cols":
+        packed = torch.zeros((packed.shape[0], packed.shape[1] - 4), dtype=torch.int32)
+    elif bad == "scales_transposed":
+        s = torch.zeros((128, 256 // g), dtype=torch.float16)
+    elif bad == "zeros_shape":
+        z = torch.zeros((1, 128), dtype=torch.float16)
+    elif bad == "out_shape":
+        out = torch.zeros((16, 120), dtype=torch.bfloat16)
+    elif bad == "x_1d":
+        x = torch.zeros(16 * 256, dtype=torch.bfloat16)
+    elif bad == "packed_dtype":
+        packed = packed.to(torch.int64)
+    elif bad == "x_noncontig":
+        x = torch.zeros((256, 16), dtype=torch.bfloat16).t()
+    with pytest.raises(ValueError, match=match):
+        lb.gemm(x, packed, s, z, bits, g, out=out)
+
+
+def test_binding_rejects_cpu_tensors_and_bad_descs():
+    x, packed, s, z = _cpu_args()
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        lb.gemm(x, packed, s, z, 2, 128)
+    import torch
+    y = torch.zeros((16, 128), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        lb.make_desc(x, packed, s, z, y, 2, 128)
+    with pytest.raises(ValueError, match="out: expected shape"):
+        lb.make_desc(x, packed, s, z, torch.zeros((16, 64), dtype=torch.bfloat16), 2, 128)
+    with pytest.raises(ValueError, match="packed: 8 words"):
+        lb.unpack(torch.zeros((2, 4), dtype=torch.int32), 4, 64, 2)

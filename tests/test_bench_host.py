@@ -90,8 +90,8 @@ def test_reference_arm_prints_contract_line_on_rank0():
 
 
 def test_reference_arm_other_ranks_exit_quietly():
-    r = _run_bench(["--impl", "reference", "--workload", "tiny_ternary_g64", "--steps", "1", "--warmup", "3"],
-                   {"RANK": "1", "WORLD_SIZE": "2"})
+    r = _run_bench(["--impl", "reference", "--workload", "tiny_ternary_g64", "--steps", "1", "--warmup", "3",
+                    "--gpus", "2"], {"RANK": "1", "WORLD_SIZE": "2"})
     assert r.returncode == 0, r.stderr
     assert r.stdout.strip() == ""
 
@@ -119,3 +119,23 @@ def test_measured_traffic_follows_the_kernel_sources(tmp_path, monkeypatch):
     assert bench.kernel_source_hash() != h
     assert bench.measured_traffic("w") is None          # a changed kernel invalidates the capture
 
+
+def test_gpus_flag_launches_that_many_ranks():
+    """`--gpus 2` outside torchrun starts two ranks itself (torchrun on 127.0.0.1): rank 0 prints the
+    one line, with n_gpus equal to the ranks that ran; the other rank prints nothing."""
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK", "MASTER_ADDR",
+                                                             "MASTER_PORT")}
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
+                        "--workload", "tiny_ternary_g64", "--steps", "1", "--warmup", "3", "--ref-rows", "4"],
+                       capture_output=True, text=True, env=env, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    line = json.loads(lines[0])
+    assert line["n_gpus"] == 2 and line["impl"] == "reference"
+
+
+def test_world_must_match_gpus():
+    bench.check_world(2, 2)
+    with pytest.raises(SystemExit):
+        bench.check_world(4, 2)

@@ -1,8 +1,11 @@
 """GPU GEMM against the fp64 CPU oracle.
 
 Bound per element: |gpu - ref| <= 1e-2 |ref| + 1e-2 rms(ref) (ref = oracle, fp64). Small and
-ragged shapes are compared whole; full workload sizes are compared on sampled entries (4096
-random ones plus 16 full rows and 16 full columns) in the configuration the benchmark runs.
+ragged shapes are compared whole, and so are the full-size ternary QKV linear at a 512x512 image
+and the text-encoder linears at 512 and 16 tokens. The 1024x1024 binary MLP linears and the
+denoise-step chain are compared on sampled entries (4096 random ones plus 16 full rows and 16
+full columns per shape), and the step's 80-linear batch call is sampled linear by linear as the
+benchmark runs it.
 """
 import numpy as np
 import pytest
@@ -117,6 +120,50 @@ def test_gemm_small_m_warp_mma(bits, gs, M, K, N, rows, ksplit):
     _gpu.check_close(_gpu.y_to_f64(y), ref, what=f"warp-mma M={M} K={K} N={N} rows={rows} split={ksplit}")
 
 
+@pytest.mark.parametrize("bits,gs", FORMATS)
+@pytest.mark.parametrize("M", [1, 3, 8])
+@pytest.mark.parametrize("K,N,rows,ksplit", [
+    (256, 520, 0, 1),       # one step, half of it past K
+    (768, 264, 0, 3),       # a request for 3 slices served with 2
+    (2560, 1032, 0, 0),     # automatic choice
+    (9728, 256, 0, 0),      # long K, few rows: split over a cluster
+    (640, 136, 48, 0),      # 3 units of 16 rows, the last tile half past N
+    (1152, 1000, 112, 2),   # the second slice holds one 128-wide group of K
+    (1024, 2376, 16, 1),    # more row blocks than SMs: persistent tiles, no cluster
+    (2048, 1352, 16, 2),    # persistent tiles with the cross-rank reduction on every tile
+])
+def test_gemm_small_m_weights_as_16_row_operand(bits, gs, M, K, N, rows, ksplit):
+    """The small-M kernel with weights as the MMA's 16-row operand and at most 8 tokens as its n8
+    operand (tile_tokens = 8, the automatic choice for M <= 8): ragged N and K, forced tilings."""
+    if bits == 1 and K % 128:
+        pytest.skip("binary needs K % 128 == 0")
+    spec = spec_for(bits, gs, M, K, N, seed=M * 11 + K)
+    prob = synth.make_problem(spec)
+    ref = oracle.gemm(prob.x_bf16, _gpu.oracle_packed(prob), prob.scales, prob.zeros, N, bits, gs)
+    x, packed, s, z = _gpu.dev_problem(prob)
+    y = lb.gemm(x, packed, s, z, bits, gs, tile_tokens=8, tile_rows=rows, ksplit=ksplit)
+    torch.cuda.synchronize()
+    assert lb.device_status() == 0
+    _gpu.check_close(_gpu.y_to_f64(y), ref, what=f"weights-as-A M={M} K={K} N={N} rows={rows} split={ksplit}")
+
+
+@pytest.mark.parametrize("bits,gs", [(2, 128), (4, 64)])
+def test_small_m_orientations_agree_and_auto_picks_weights_as_a(bits, gs):
+    """At M <= 8 both orientations compute the same products; the automatic configuration is the
+    weights-as-A kernel (bit-identical to tile_tokens = 8)."""
+    spec = spec_for(bits, gs, 6, 3072, 1032, seed=81)
+    prob = synth.make_problem(spec)
+    ref = oracle.gemm(prob.x_bf16, _gpu.oracle_packed(prob), prob.scales, prob.zeros, spec.N, bits, gs)
+    x, packed, s, z = _gpu.dev_problem(prob)
+    y_auto = lb.gemm(x, packed, s, z, bits, gs)
+    y8 = lb.gemm(x, packed, s, z, bits, gs, tile_tokens=8)
+    y16 = lb.gemm(x, packed, s, z, bits, gs, tile_tokens=1)
+    torch.cuda.synchronize()
+    assert torch.equal(y_auto.view(torch.int16), y8.view(torch.int16))
+    for y in (y8, y16):
+        _gpu.check_close(_gpu.y_to_f64(y), ref, what="orientation")
+
+
 def test_gemm_small_m_deterministic():
     """Repeated small-M runs with a cluster split give bit-identical outputs (fixed summation order)."""
     spec = spec_for(4, 64, 16, 9728, 2560, seed=5)
@@ -153,21 +200,76 @@ def test_all_zero_ternary_gives_zero():
     assert torch.count_nonzero(y.float()) == 0
 
 
+def integer_problem(bits, M, K, N, g, seed, nonzeros=None):
+    """Unit scales, integer zeros (8), codes with |w| <= 1 and x in {-1,0,1} with at most
+    `nonzeros` (default K) nonzero entries per row: every product and partial sum is an integer
+    and |y| <= 256, so the exact result is a bf16 value."""
+    codes = _pins.random_codes(N, K, bits, seed=seed)
+    if bits == 4:
+        codes = np.random.default_rng(seed).integers(7, 10, size=(N, K)).astype(np.int8)
+    x = _pins.x_as_f64(_pins.small_int_x(M, K, seed=seed))
+    if nonzeros is not None:
+        r = np.random.default_rng(seed + 1)
+        for m in range(M):
+            x[m, r.permutation(K)[nonzeros:]] = 0.0
+    x = _pins.bf16_bits_from_f32(x.astype(np.float32))
+    s = np.ones((K // g, N), dtype=np.float16)
+    z = np.full((K // g, N), 8.0, dtype=np.float16) if bits == 4 else None
+    return synth.Problem(spec_for(bits, g, M, K, N), x, codes, s, z)
+
+
 @pytest.mark.parametrize("bits", [1, 2, 4])
 def test_integer_exact(bits):
     """Unit scales, integer zeros, x in {-1,0,1}, |y| <= 256: bf16 output equals the oracle."""
     M, N, K, g = 70, 136, 256, 64
-    codes = _pins.random_codes(N, K, bits, seed=bits)
-    if bits == 4:
-        codes = np.random.default_rng(bits).integers(7, 10, size=(N, K)).astype(np.int8)
-    x = _pins.small_int_x(M, K, seed=bits)
-    s = np.ones((K // g, N), dtype=np.float16)
-    z = np.full((K // g, N), 8.0, dtype=np.float16) if bits == 4 else None
-    prob = synth.Problem(spec_for(bits, g, M, K, N), x, codes, s, z)
-    ref = oracle.gemm(x, _gpu.oracle_packed(prob), s, z, N, bits, g)
+    prob = integer_problem(bits, M, K, N, g, seed=bits)
+    ref = oracle.gemm(prob.x_bf16, _gpu.oracle_packed(prob), prob.scales, prob.zeros, N, bits, g)
     xd, packed, sd, zd = _gpu.dev_problem(prob)
     y = _gpu.y_to_f64(lb.gemm(xd, packed, sd, zd, bits, g))
     assert np.array_equal(y, ref)
+
+
+@pytest.mark.parametrize("bits", [1, 2, 4])
+@pytest.mark.parametrize("M,tile_tokens", [(1, 1), (5, 1), (16, 1), (1, 8), (5, 8), (8, 8)])
+@pytest.mark.parametrize("K,nonzeros,ksplit", [(256, None, 1), (2048, 256, 2), (1024, 200, 0)])
+def test_integer_exact_small_m(bits, M, tile_tokens, K, nonzeros, ksplit):
+    """The small-M kernel on integer problems: it decodes codes without their scale (+-1, 128 + f,
+    128 + q), sums one group at a time in fp32 and subtracts c * Sx, so every intermediate is an
+    exact integer and the bf16 output must equal the oracle bit for bit -- also across the
+    cluster's K split (ksplit 2) and the automatic tiling, in both orientations (X or the weights
+    as the 16-row MMA operand)."""
+    N, g = 264, 64
+    if bits == 1 and K % 128:
+        pytest.skip("binary needs K % 128 == 0")
+    prob = integer_problem(bits, M, K, N, g, seed=10 * bits + M, nonzeros=nonzeros)
+    ref = oracle.gemm(prob.x_bf16, _gpu.oracle_packed(prob), prob.scales, prob.zeros, N, bits, g)
+    assert np.abs(ref).max() <= 256
+    xd, packed, sd, zd = _gpu.dev_problem(prob)
+    y = _gpu.y_to_f64(lb.gemm(xd, packed, sd, zd, bits, g, tile_tokens=tile_tokens, ksplit=ksplit))
+    torch.cuda.synchronize()
+    assert lb.device_status() == 0
+    assert np.array_equal(y, ref)
+
+
+@pytest.mark.parametrize("M,tile_tokens", [(96, 0), (300, 0), (16, 1), (16, 16), (5, 1), (5, 8)])
+def test_uint4_codes_at_their_zero_point(M, tile_tokens):
+    """uint4 codes equal or next to their group's zero point, with zero points that are not
+    integers: each weight (q - z) * s is a small difference of two large terms. The
+    tensor-memory kernel rounds every weight once to fp16 from its exact value (the small-M
+    kernel sums exact codes and subtracts (128 + z) * s * Sx in fp32), so the outputs stay
+    inside the tolerance although every |w| is far below |z * s|."""
+    N, K, g = 264, 1024, 64
+    r = np.random.default_rng(M + tile_tokens)
+    q0 = r.integers(6, 10, size=(K // g, N))                           # per group
+    dz = r.choice([-3, -2, -1, 1, 2, 3], size=(K // g, N)) / 128.0      # z = q0 + dz, fp16-exact
+    z = (q0 + dz).astype(np.float16)
+    assert np.array_equal(z.astype(np.float64), q0 + dz)
+    step = r.choice([-1, 0, 0, 0, 1], size=(N, K))                      # codes mostly equal to q0
+    codes = np.clip(np.repeat(q0.T, g, axis=1) + step, 0, 15).astype(np.int8)
+    spec = spec_for(4, g, M, K, N, seed=77)
+    prob = synth.make_problem(spec)
+    prob = synth.Problem(spec, prob.x_bf16, codes, prob.scales, z)
+    run_and_compare(spec, tile_tokens=tile_tokens, prob=prob)
 
 
 def test_orientation_square():
@@ -216,11 +318,23 @@ def sampled_check(spec, seed=0, n_random=4096, n_rows=16, n_cols=16):
     return _gpu.check_close(y[ms, ns], ref, rms=rms, what=spec.name)
 
 
-FULL = [s for w in ("qkv_512sq_ternary_g128", "mlp_1024sq_binary_g128", "te_m512_uint4_g64", "te_m16_uint4_g64")
-        for s in synth.WORKLOADS[w]]
+FULL_WHOLE = [s for w in ("qkv_512sq_ternary_g128", "te_m512_uint4_g64", "te_m16_uint4_g64",
+                           *(f"klein_linears_m{m}_{f}_g128" for f in ("ternary", "binary") for m in (1, 4, 16)))
+              for s in synth.WORKLOADS[w]]
+FULL_SAMPLED = synth.WORKLOADS["mlp_1024sq_binary_g128"]
 
 
-@pytest.mark.parametrize("spec", FULL, ids=lambda s: s.name)
+@pytest.mark.parametrize("spec", FULL_WHOLE, ids=lambda s: s.name)
+def test_full_size_whole(spec):
+    """The ternary QKV linear at a 512x512 image (1536 x 3072 -> 9216), the uint4 text-encoder
+    linears at 512 and 16 tokens and the transformer's ternary / binary linear shapes at 1, 4 and
+    16 tokens, every output element against the oracle."""
+    y, ref = run_and_compare(spec)
+    worst = _gpu.check_close(_gpu.y_to_f64(y), ref, what=spec.name)
+    print(f"\n{spec.name} M={spec.M} K={spec.K} N={spec.N}: max err/bound {worst:.3f} over all {ref.size}")
+
+
+@pytest.mark.parametrize("spec", FULL_SAMPLED, ids=lambda s: s.name)
 def test_full_size_sampled(spec):
     worst = sampled_check(spec)
     print(f"\n{spec.name} M={spec.M} K={spec.K} N={spec.N}: max err/bound {worst:.3f}")
@@ -256,8 +370,49 @@ def chain_distinct():
 
 @pytest.mark.parametrize("spec", chain_distinct(), ids=lambda s: s.name)
 def test_chain_shapes_sampled(spec):
-    worst = sampled_check(spec, n_random=2048, n_rows=4, n_cols=4)
+    worst = sampled_check(spec)
     print(f"\n{spec.name} M={spec.M} K={spec.K} N={spec.N}: max err/bound {worst:.3f}")
+
+
+def sample_entries(M, N, r, n_random, n_rows, n_cols):
+    """Random (m, n) entries plus every entry of a few full rows and full columns."""
+    ms = [r.integers(0, M, n_random)]
+    ns = [r.integers(0, N, n_random)]
+    for m in r.choice(M, size=min(n_rows, M), replace=False):
+        ms.append(np.full(N, m))
+        ns.append(np.arange(N))
+    for n in r.choice(N, size=min(n_cols, N), replace=False):
+        ms.append(np.arange(M))
+        ns.append(np.full(M, n))
+    return np.concatenate(ms), np.concatenate(ns)
+
+
+def test_chain_batch_as_run_sampled():
+    """The headline call as the benchmark makes it: one lowbit_gemm_batch over the 80 linears of
+    a denoise step at a 1024x1024 image (weights packed on the GPU, outputs pre-filled with NaN),
+    then every linear's output sampled against the oracle (1024 random entries, 2 full rows and
+    2 full columns each; each distinct shape is also checked more densely above)."""
+    specs = synth.chain_linears()
+    dev = []
+    for sp in specs:
+        x, packed, s, z = _gpu.dev_problem(synth.make_problem(sp))
+        y = torch.full((sp.M, sp.N), float("nan"), dtype=torch.bfloat16, device="cuda")
+        dev.append((x, packed, s, z, y))
+    descs = [lb.make_desc(x, w, s, z, y, sp.bits, sp.group_size) for sp, (x, w, s, z, y) in zip(specs, dev)]
+    lb.gemm_batch(descs)
+    torch.cuda.synchronize()
+    assert lb.device_status() == 0
+    r = np.random.default_rng(80)
+    worst = 0.0
+    for sp, (_, _, _, _, y) in zip(specs, dev):
+        prob = synth.make_problem(sp)
+        ms, ns = sample_entries(sp.M, sp.N, r, 1024, 2, 2)
+        got = y[torch.from_numpy(ms).cuda(), torch.from_numpy(ns).cuda()].float().cpu().numpy().astype(np.float64)
+        ref = oracle.gemm_entries(prob.x_bf16, _gpu.oracle_packed(prob), prob.scales, prob.zeros, sp.N, sp.bits,
+                                  sp.group_size, ms, ns)
+        rms = float(np.sqrt(np.mean(ref * ref)))
+        worst = max(worst, _gpu.check_close(got, ref, rms=rms, what=sp.name))
+    print(f"\n80-linear batch: max err/bound {worst:.3f}")
 
 
 def test_batch_matches_single_calls():
@@ -290,6 +445,39 @@ def test_batch_chain_dependency():
     want = lb.gemm(lb.gemm(xa, wa, sa, None, 2, 128), wb, sb, None, 2, 128)
     torch.cuda.synchronize()
     assert torch.equal(yb, want)
+
+
+def test_batch_reuses_x_copy_only_while_x_is_unchanged():
+    """Q, K and V of one input in one batch: the X conversion runs once and every output matches
+    its single call bit for bit. Then a linear whose output overwrites that X sits between two
+    readers of it: the second reader must see the new contents (the copy is made again)."""
+    M, K = 96, 512
+    specs = [spec_for(2, 128, M, K, n, seed=60 + i) for i, n in enumerate((264, 136, 512))]
+    probs = [synth.make_problem(sp) for sp in specs]
+    x, _, _, _ = _gpu.dev_problem(probs[0])
+    ws = [_gpu.dev_problem(p)[1:] for p in probs]
+    outs = [torch.empty((M, sp.N), dtype=torch.bfloat16, device="cuda") for sp in specs]
+    descs = [lb.make_desc(x, w, s, z, y, 2, 128) for (w, s, z), y in zip(ws, outs)]
+    lb.gemm_batch(descs)
+    singles = [lb.gemm(x, w, s, z, 2, 128) for (w, s, z) in ws]
+    torch.cuda.synchronize()
+    for sp, y1, y2 in zip(specs, outs, singles):
+        assert torch.equal(y1.view(torch.int16), y2.view(torch.int16)), sp.name
+    # reader, writer of X (K -> N = K, so its output has X's shape), reader again
+    wspec = spec_for(2, 128, M, K, K, seed=70)
+    wprob = synth.make_problem(wspec)
+    x2, w2, s2, _ = _gpu.dev_problem(wprob)
+    xa = x.clone()
+    ya, yb = torch.empty_like(outs[0]), torch.empty_like(outs[0])
+    (w0, s0, _) = ws[0]
+    lb.gemm_batch([lb.make_desc(xa, w0, s0, None, ya, 2, 128), lb.make_desc(x2, w2, s2, None, xa, 2, 128),
+                   lb.make_desc(xa, w0, s0, None, yb, 2, 128)])
+    want_x = lb.gemm(x2, w2, s2, None, 2, 128)
+    want_b = lb.gemm(want_x, w0, s0, None, 2, 128)
+    torch.cuda.synchronize()
+    assert torch.equal(ya.view(torch.int16), singles[0].view(torch.int16))
+    assert torch.equal(xa.view(torch.int16), want_x.view(torch.int16))
+    assert torch.equal(yb.view(torch.int16), want_b.view(torch.int16))
 
 
 def test_bounded_wait_timeout_is_reported():
@@ -326,11 +514,12 @@ def test_extreme_row_magnitudes():
 
 
 @pytest.mark.parametrize("bits,gs", [(1, 128), (2, 128), (4, 64)])
-def test_small_m_row_magnitudes(bits, gs):
+@pytest.mark.parametrize("M,tile_tokens", [(9, 1), (8, 8)])
+def test_small_m_row_magnitudes(bits, gs, M, tile_tokens):
     """The small-M kernel sums unscaled codes times X in fp32 per group, so it is exact for
     |x| up to about 2^114; rows scaled by 2^100 and 2^-100, tiny and zero rows match the oracle
     row by row."""
-    spec = spec_for(bits, gs, 9, 1024, 264, seed=41)
+    spec = spec_for(bits, gs, M, 1024, 264, seed=41)
     prob = synth.make_problem(spec)
     x = _pins.x_as_f64(prob.x_bf16)
     x[0] *= 2.0 ** 100
@@ -341,7 +530,7 @@ def test_small_m_row_magnitudes(bits, gs):
     prob.x_bf16 = _pins.bf16_bits_from_f32(x.astype(np.float32))
     ref = oracle.gemm(prob.x_bf16, _gpu.oracle_packed(prob), prob.scales, prob.zeros, spec.N, bits, gs)
     xd, packed, s, z = _gpu.dev_problem(prob)
-    y = _gpu.y_to_f64(lb.gemm(xd, packed, s, z, bits, gs, tile_tokens=1))
+    y = _gpu.y_to_f64(lb.gemm(xd, packed, s, z, bits, gs, tile_tokens=tile_tokens))
     torch.cuda.synchronize()
     assert np.all(y[2] == 0.0)
     for m in range(spec.M):
