@@ -311,7 +311,9 @@ def run_lowbit(args, specs, workload):
     peaks, peak_src = load_peaks()
     # bound of the workload: below the ridge point (peak flop/s per peak byte/s) it is HBM-bound
     hbm_bound = is_hbm_bound(flops, nbytes, peaks)
-    launches_per_step = sum(1 if s.M <= 16 else 2 for s in specs)   # X conversion + GEMM above 16 tokens
+    # kernels per step: one per linear of at most 16 tokens, two above (X conversion + GEMM; every
+    # linear here has its own X)
+    launches_per_step = sum(1 if s.M <= 16 else 2 for s in specs)
 
     def barrier():
         if world > 1:

@@ -84,9 +84,16 @@ struct Choice {
     int rows, ksplit, kslice, clusters;
 };
 
-// Rows per CTA and K slices: the fewest waves of the largest per-CTA share (rows x K slice),
-// rows counted at least 48 since fewer leave too few MMA chains to cover their latency. Rows
-// come in multiples of `align` (8, or 16 with weights as the 16-row operand).
+// Time model of the kernel, fitted to B200 measurements at 16 tokens (microseconds): a 512-wide
+// K step of a CTA costs a + b * rows (a: the step's fixed work -- waiting for the ring, the X
+// fragments, group sums and scale table, the refill -- b: decode, MMAs and scaling per row), and
+// summing K slices across a cluster about 2 us per row block. Long-K runs gave a = 0.64 /
+// b = 0.0072 for uint4 and 0.41 / 0.0086 for ternary; binary uses the ternary figures.
+double step_us(int bits, int rows) { return bits == 4 ? 0.64 + 0.0072 * rows : 0.41 + 0.0086 * rows; }
+constexpr double kSplitUs = 2.0;
+
+// Rows per CTA (a multiple of `align`: 8, or 16 with weights as the 16-row operand) and K slices
+// with the smallest modelled time: waves x (steps per slice x step time + the split's reduction).
 Choice choose(const void* probe, int bits, int gs, int N, int K, int force_rows, int force_split, bool swap) {
     const int align = swap ? 16 : 8;
     Choice best{0, 0, 0, 0};
@@ -97,18 +104,20 @@ Choice choose(const void* probe, int bits, int gs, int N, int K, int force_rows,
         const int ks_eff = (K + kslice - 1) / kslice;
         if (!force_split && ks_eff != ks) continue;
         const int cap = cluster_capacity(probe, bits, gs, ks_eff, swap);
-        int rows = force_rows;
-        if (!rows) {
-            rows = align * ((N + align * cap - 1) / (align * cap));
-            if (rows < align) rows = align;
-            if (rows > kMaxRows) rows = kMaxRows;
-        }
-        const int nb = (N + rows - 1) / rows;
-        const int waves = (nb + cap - 1) / cap;
-        const double cost = static_cast<double>(waves) * (rows < 48 ? 48 : rows) * kslice;
-        if (!best.rows || cost < best_cost) {
-            best = Choice{rows, ks_eff, kslice, nb < cap ? nb : cap};
-            best_cost = cost;
+        int fit = align * ((N + align * cap - 1) / (align * cap));   // rows that spread N over every cluster
+        if (fit < align) fit = align;
+        if (fit > kMaxRows) fit = kMaxRows;
+        const int cands[5] = {force_rows ? force_rows : fit, 64, 96, 128, 48};
+        for (int c = 0; c < (force_rows ? 1 : 5); ++c) {
+            const int rows = cands[c];
+            if (rows % align || rows > kMaxRows) continue;
+            const int nb = (N + rows - 1) / rows;
+            const int waves = (nb + cap - 1) / cap;
+            const double cost = waves * ((kslice / kStepK) * step_us(bits, rows) + (ks_eff > 1 ? kSplitUs : 0.0));
+            if (!best.rows || cost < best_cost) {
+                best = Choice{rows, ks_eff, kslice, nb < cap ? nb : cap};
+                best_cost = cost;
+            }
         }
     }
     return best;

@@ -241,11 +241,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     grid_launch_dependents();
 
     // Ring step `gs` of this CTA: tile blockIdx.x + (gs / nst) * gridDim.x, K step gs % nst.
+    // Every CTA of a slice reads the same X (only its weight rows differ). Walking the slice's K
+    // steps from a different first step per CTA spreads those reads over the whole slice, instead
+    // of every SM asking the same few L2 lines for the same 16 KB at the same moment. (Each CTA's
+    // summation order is still fixed, so results stay run-to-run identical.)
+    const int rot = static_cast<int>(blockIdx.x) % nst;
     auto issue = [&](int gs, bool codes, bool x) {
         const int s = gs % S;
         uint8_t* st = ring + s * p.stage_bytes;
         const int n0 = (static_cast<int>(blockIdx.x) + (gs / nst) * static_cast<int>(gridDim.x)) * R;
-        const int kk = k_begin + (gs % nst) * kStepK;
+        int kc = gs % nst + rot;
+        if (kc >= nst) kc -= nst;
+        const int kk = k_begin + kc * kStepK;
         if (codes) {
             mbar_arrive_expect_tx(&full[s], p.tx_bytes);
 #pragma unroll

@@ -139,3 +139,4 @@ def test_world_must_match_gpus():
     bench.check_world(2, 2)
     with pytest.raises(SystemExit):
         bench.check_world(4, 2)
+
