@@ -240,10 +240,15 @@ def cpu_baseline(specs, rows_per_shape=32):
     sample = oracle_sample(specs, rows_per_shape)
     flops, dt = time_oracle(sample)
     nshapes = len(sample)
+    # the tiny configuration (64 x 256 x 512, ternary g64) whole, on one thread
+    tiny = oracle_sample(synth.WORKLOADS["tiny_ternary_g64"], 64)
+    tf, t1 = time_oracle(tiny, threads=1)
     return {"value": flops / dt / 1e12, "unit": UNIT, "cores": oracle.default().threads(0), "kind": "oracle",
             "sample": f"{nshapes} distinct shapes of the workload, first {rows_per_shape} activation rows each "
                       f"(full K and N, weights decoded inside the timed call); {flops / 1e9:.1f} GFLOP in {dt:.1f} s",
-            "host_cpus": os.cpu_count()}
+            "host_cpus": os.cpu_count(),
+            "single_thread_tiny": {"seconds": t1, "tflops": tf / t1 / 1e12,
+                                   "what": "the whole 64 x 256 x 512 ternary g64 GEMM on one host thread"}}
 
 
 # --------------------------------------------------------------------------------------------
@@ -513,7 +518,9 @@ def run_lowbit(args, specs, workload):
         achieved = launch_bytes / (launch_ms * 1e-3) / 1e9
         roofline = {"bound": "hbm", "achieved": achieved, "peak": peak_bw, "unit": "GB/s",
                     "frac": achieved / peak_bw, "traffic": traffic,
-                    "peak_source": f"{peak_src} HBM copy bandwidth", "kernel": "lowbit_smallm_kernel",
+                    "peak_source": f"{peak_src} HBM copy bandwidth",
+                    "kernel": ("lowbit_smallm_kernel" if all(sp.M <= 16 for sp in specs)
+                               else "lowbit_gemm_kernel (+ X conversion), one lowbit_gemm call"),
                     "us_per_launch": launch_ms * 1e3, "launches_timed": launches_timed,
                     "algorithmic_mb_per_launch": launch_bytes / 1e6,
                     "algorithmic_gflop_per_launch": launch_flops / 1e9,
