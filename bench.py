@@ -81,6 +81,104 @@ def is_hbm_bound(flops: float, nbytes: float, peaks: dict) -> bool:
     return flops / nbytes < ridge
 
 
+def measure_shapes(items, copies, lb, torch, device, stream, cap_stream, samples=9, replays=5):
+    """Per-launch durations of each distinct shape of `items` (ms): {(M, K, N): (call, GEMM kernel,
+    X conversion, reps)}.
+
+    For each distinct shape, graph A holds `reps` back-to-back lowbit_gemm calls (rotating weight
+    copies where there are several, so weights stream from HBM as in the timed steps) and graph B
+    one lowbit_gemm_batch of the same `reps` linears sharing one X, which the library converts
+    once. A sample replays a graph `replays` times between two events on the launching stream; the
+    per-launch time is the median over `samples` samples of sample time / (replays * reps). For
+    more than 16 tokens a call is the X conversion pass plus the GEMM kernel: the conversion's time
+    is (A - B) / (reps - 1) per launch and the GEMM kernel's is the call's minus that. At most 16
+    tokens a call is the small-M GEMM kernel alone."""
+    def time_graph(gph, per_sample, warm=2):
+        for _ in range(warm):
+            gph.replay()
+        torch.cuda.synchronize(device)
+        ts = []
+        for _ in range(samples):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(replays):
+                gph.replay()
+            e1.record(stream)
+            torch.cuda.synchronize(device)
+            ts.append(e0.elapsed_time(e1) / (replays * per_sample))
+        return statistics.median(ts)
+
+    def capture(fn):
+        gph = torch.cuda.CUDAGraph()
+        cap_stream.wait_stream(stream)
+        with torch.cuda.stream(cap_stream):
+            with torch.cuda.graph(gph, stream=cap_stream):
+                fn()
+        stream.wait_stream(cap_stream)
+        return gph
+
+    shape_times = {}
+    seen = {}
+    for it in items:
+        seen.setdefault((it["spec"].M, it["spec"].K, it["spec"].N), it)
+    for key, it in seen.items():
+        reps = max(10, copies)
+        sp = it["spec"]
+
+        def calls():
+            for i in range(reps):
+                w_p, w_s, w_z = it["reps"][i % copies]
+                lb.gemm(it["x"], w_p, w_s, w_z, sp.bits, sp.group_size, out=it["y"])
+
+        g_a = capture(calls)
+        t_call = time_graph(g_a, reps)
+        del g_a
+        t_conv = 0.0
+        if sp.M > 16:
+            shared = [lb.make_desc(it["x"], *it["reps"][i % copies], it["y"], sp.bits, sp.group_size)
+                      for i in range(reps)]
+            g_b = capture(lambda: lb.gemm_batch(shared, device))
+            t_shared = time_graph(g_b, reps)
+            del g_b
+            t_conv = max(0.0, (t_call - t_shared) * reps / (reps - 1))
+        shape_times[key] = (t_call, t_call - t_conv, t_conv, reps)
+    return shape_times
+
+
+CONFIGS = ("tiny_ternary_g64", "qkv_512sq_ternary_g128", "mlp_1024sq_binary_g128", "te_m512_uint4_g64",
+           "te_m16_uint4_g64", "klein_linears_m1_ternary_g128")
+
+
+def measure_configs(lb, torch, device, stream, cap_stream, peaks, l2_bytes):
+    """Per-launch results of the reference configurations (see CONFIGS), each linear timed as in
+    measure_shapes with fewer samples: per shape the call, GEMM kernel and conversion times, the
+    throughput of the GEMM kernel and its fraction of the burst bf16 peak (tensor-bound) or of the
+    HBM bandwidth (HBM-bound)."""
+    out = {}
+    for name in CONFIGS:
+        specs = synth.WORKLOADS[name]
+        copies = rotation_copies(step_bytes(specs), weight_bytes(specs), l2_bytes)
+        items, _ = setup(specs, device, lb, torch, pinned=False, copies=copies)
+        times = measure_shapes(items, copies, lb, torch, device, stream, cap_stream, samples=5, replays=3)
+        hbm = is_hbm_bound(step_flops(specs), step_bytes(specs), peaks)
+        shapes = []
+        for sp in specs:
+            t_call, t_gemm, t_conv, _ = times[(sp.M, sp.K, sp.N)]
+            e = {"MKN": [sp.M, sp.K, sp.N], "call_us": t_call * 1e3, "gemm_us": t_gemm * 1e3,
+                 "x_conversion_us": t_conv * 1e3, "gemm_tflops": sp.flops / (t_gemm * 1e-3) / 1e12,
+                 "call_gbs": sp.algorithmic_bytes() / (t_call * 1e-3) / 1e9}
+            if hbm:
+                e["frac_of_hbm"] = e["call_gbs"] / peaks.get("hbm_gbs")
+            else:
+                e["gemm_frac_of_burst"] = e["gemm_tflops"] / peaks.get("bf16_tflops")
+            shapes.append(e)
+        out[name] = {"bound": "hbm" if hbm else "tensor", "weight_copies_rotated": copies, "linears": shapes}
+        del items
+        torch.cuda.synchronize(device)
+        torch.cuda.empty_cache()
+    return out
+
+
 def max_over_ranks(v: float, world: int, device=None) -> float:
     """The maximum of v over all ranks of the default process group (v itself when alone)."""
     if world == 1:
@@ -374,64 +472,7 @@ def run_lowbit(args, specs, workload):
     if lb.device_status() != 0:
         raise RuntimeError("kernel timeout reported during the timed steps")
 
-    # Per-launch durations for the roofline. For each distinct shape, graph A holds `reps`
-    # back-to-back lowbit_gemm calls (rotating weight copies where there are several, so weights
-    # stream from HBM as in the timed steps) and graph B one lowbit_gemm_batch of the same `reps`
-    # linears sharing one X, which the library converts once. A sample replays a graph
-    # `replays` times between two events on the launching stream; the per-launch time is the
-    # median over samples of sample time / (replays * reps). For more than 16 tokens a call is
-    # the X conversion pass plus the GEMM kernel: the conversion's time is (A - B) / (reps - 1)
-    # per launch and the GEMM kernel's is the call's minus that. At most 16 tokens a call is the
-    # small-M GEMM kernel alone.
-    def time_graph(gph, per_sample, samples=9, replays=5, warm=2):
-        for _ in range(warm):
-            gph.replay()
-        torch.cuda.synchronize(device)
-        ts = []
-        for _ in range(samples):
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            for _ in range(replays):
-                gph.replay()
-            e1.record(stream)
-            torch.cuda.synchronize(device)
-            ts.append(e0.elapsed_time(e1) / (replays * per_sample))
-        return statistics.median(ts)
-
-    def capture(fn):
-        gph = torch.cuda.CUDAGraph()
-        cap_stream.wait_stream(stream)
-        with torch.cuda.stream(cap_stream):
-            with torch.cuda.graph(gph, stream=cap_stream):
-                fn()
-        stream.wait_stream(cap_stream)
-        return gph
-
-    shape_times = {}
-    seen = {}
-    for it in items:
-        seen.setdefault((it["spec"].M, it["spec"].K, it["spec"].N), it)
-    for key, it in seen.items():
-        reps = max(10, copies)
-        sp = it["spec"]
-
-        def calls():
-            for i in range(reps):
-                w_p, w_s, w_z = it["reps"][i % copies]
-                lb.gemm(it["x"], w_p, w_s, w_z, sp.bits, sp.group_size, out=it["y"])
-
-        g_a = capture(calls)
-        t_call = time_graph(g_a, reps)
-        del g_a
-        t_conv = 0.0
-        if sp.M > 16:
-            shared = [lb.make_desc(it["x"], *it["reps"][i % copies], it["y"], sp.bits, sp.group_size)
-                      for i in range(reps)]
-            g_b = capture(lambda: lb.gemm_batch(shared, device))
-            t_shared = time_graph(g_b, reps)
-            del g_b
-            t_conv = max(0.0, (t_call - t_shared) * reps / (reps - 1))
-        shape_times[key] = (t_call, t_call - t_conv, t_conv, reps)
+    shape_times = measure_shapes(items, copies, lb, torch, device, stream, cap_stream)
     per = [(s, *shape_times[(s.M, s.K, s.N)][:3]) for s in specs]     # (spec, call, gemm, conversion) ms
     launch_ms = sum(c for _, c, _, _ in per) / len(per)
     gemm_ms = sum(g for _, _, g, _ in per) / len(per)
@@ -439,6 +480,11 @@ def run_lowbit(args, specs, workload):
     launch_flops = sum(sp.flops for sp, _, _, _ in per) / len(per)
     launch_bytes = sum(sp.algorithmic_bytes() for sp, _, _, _ in per) / len(per)
     launches_timed = sum(2 * 9 * 5 * r if k[0] > 16 else 9 * 5 * r for k, (_, _, _, r) in shape_times.items())
+    # Per-launch figures of the other reference configurations, measured the same way after the
+    # headline's timed region (so that one run of the default workload corroborates them).
+    others = None
+    if world == 1 and not args.no_configs and workload == DEFAULT_WORKLOAD:
+        others = measure_configs(lb, torch, device, stream, cap_stream, peaks, l2_bytes)
 
     # End to end through the public API, as a user would pipeline it: each step copies every
     # linear's activations in (pinned host -> device, copy stream), runs lowbit_gemm per linear
@@ -560,6 +606,8 @@ def run_lowbit(args, specs, workload):
                 "hbm_gbs": world * nbytes / (ms_step * 1e-3) / 1e9,
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": launches_per_step * args.steps, "clocks": clk}
+        if others is not None:
+            line["configs"] = others
         if len(specs) >= 40:   # a denoise step's chain: the pages count 4 steps per image
             line["config"]["ms_per_4_steps"] = 4 * ms_step
         print(json.dumps(line), flush=True)
@@ -607,6 +655,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--per-shape", action="store_true", help="print per-shape launch times to stderr")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the per-launch results of the other reference configurations (default workload)")
     ap.add_argument("--only-linear", default="", help="comma-separated indices of the workload's linears to run "
                                                       "(profiling one shape); default all")
     args = ap.parse_args()

@@ -314,6 +314,192 @@ __global__ void __launch_bounds__(kThreads, 1)
     float acc[NH][4];
 #pragma unroll
     for (int o = 0; o < NH; ++o) acc[o][0] = acc[o][1] = acc[o][2] = acc[o][3] = 0.f;
+
+    // ---- the phases of one ring step, shared by both loop drivers below ----
+    // P1: this warp's group: fp32 (s, s * c) of every row of its units, into `tab`
+    auto build_table = [&](const uint8_t* st, float4* tab) {
+        const __half* sh = reinterpret_cast<const __half*>(st + p.s_off) + gi * R;
+        const __half* zh = reinterpret_cast<const __half*>(st + p.z_off) + gi * R;
+        auto sc_of = [&](int r, float& sf, float& cf) {
+            sf = __half2float(sh[r]);
+            cf = BITS == 4 ? sf * (128.f + __half2float(zh[r])) : BITS == 2 ? 129.f * sf : 0.f;
+        };
+        if constexpr (SWAP) {
+            // entry 8u + g: rows 16u + g and 16u + g + 8 of the warp's units
+#pragma unroll
+            for (int i0 = 0; i0 < HP; i0 += 32) {
+                const int i = i0 + lane;
+                if (i < 8 * nh) {
+                    const int r = 16 * (ob0 + (i >> 3)) + (i & 7);
+                    float s0, c0, s1, c1;
+                    sc_of(r, s0, c0);
+                    sc_of(r + 8, s1, c1);
+                    tab[i] = make_float4(s0, s1, c0, c1);
+                }
+            }
+        } else {
+            const __half2* sp = reinterpret_cast<const __half2*>(sh) + 4 * ob0;
+            const __half2* zp = reinterpret_cast<const __half2*>(zh) + 4 * ob0;
+#pragma unroll
+            for (int i0 = 0; i0 < HP; i0 += 32) {
+                const int i = i0 + lane;
+                if (i < 4 * nh) {
+                    const float2 sf = __half22float2(sp[i]);
+                    float c0 = 0.f, c1 = 0.f;
+                    if (BITS == 4) {
+                        const float2 zf = __half22float2(zp[i]);
+                        c0 = sf.x * (128.f + zf.x);
+                        c1 = sf.y * (128.f + zf.y);
+                    } else if (BITS == 2) {
+                        c0 = 129.f * sf.x;
+                        c1 = 129.f * sf.y;
+                    }
+                    tab[i] = make_float4(sf.x, sf.y, c0, c1);
+                }
+            }
+        }
+    };
+    // P2: X fragments of this warp's four 16-wide K steps (128-byte swizzled rows): a[j] = the A
+    // operand of step j, or with SWAP a[p] = the B operands of steps 2p, 2p + 1
+    auto load_frags = [&](uint32_t st_u, uint32_t (&a)[4][4]) {
+        if constexpr (SWAP) {
+#pragma unroll
+            for (int pp = 0; pp < 2; ++pp) {
+                const int chunk = 4 * pp + (lane >> 3);
+                ldmatrix_x4(st_u + xoff + static_cast<uint32_t>((chunk ^ tok) << 4), a[pp]);
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int chunk = (j << 1) | xhalf;
+                ldmatrix_x4(st_u + xoff + static_cast<uint32_t>((chunk ^ (tok & 7)) << 4), a[j]);
+            }
+        }
+    };
+    // P3: group sums of X: tokens g (0) and g + 8 (2), or with SWAP tokens 2q (0) and 2q + 1 (1)
+    auto group_sums = [&](const uint32_t (&a)[4][4], float (&tsx)[4]) {
+        tsx[0] = tsx[1] = tsx[2] = tsx[3] = 0.f;
+        if (BITS != 1) {
+            if constexpr (SWAP) {
+                const uint32_t ones[4] = {kBf16One2, kBf16One2, kBf16One2, kBf16One2};
+                mma_bf16_z(tsx, ones, a[0][0], a[0][1]);
+                mma_bf16(tsx, ones, a[0][2], a[0][3]);
+                mma_bf16(tsx, ones, a[1][0], a[1][1]);
+                mma_bf16(tsx, ones, a[1][2], a[1][3]);
+            } else {
+                mma_bf16_z(tsx, a[0], kBf16One2, kBf16One2);
+#pragma unroll
+                for (int j = 1; j < 4; ++j) mma_bf16(tsx, a[j], kBf16One2, kBf16One2);
+            }
+        }
+    };
+    // P4: code words of the sub-batch starting at unit ob, for this warp's 64 K
+    auto load_codes = [&](const uint8_t* wst, int ob, uint32_t (&wd)[B][OPU][WPS]) {
+#pragma unroll
+        for (int u = 0; u < B; ++u) {
+            if (ob + u < nh) {
+#pragma unroll
+                for (int h = 0; h < OPU; ++h) {
+                    const uint8_t* rp = wst + (OPU * (ob0 + ob + u) + h) * kOctStride;
+                    if (BITS == 4) {
+                        wd[u][h][0] = *reinterpret_cast<const uint32_t*>(rp + wb0);
+                        wd[u][h][1] = *reinterpret_cast<const uint32_t*>(rp + wb1);
+                    } else if (BITS == 2) {
+                        wd[u][h][0] = *reinterpret_cast<const uint32_t*>(rp + wb0);
+                    } else {
+                        const uint2 v = *reinterpret_cast<const uint2*>(rp + wb0);
+                        wd[u][h][0] = v.x; wd[u][h][1] = v.y;
+                    }
+                }
+            }
+        }
+    };
+    // P5: decode + MMA chains of the sub-batch: T[u] = the unscaled group sums of unit ob + u
+    auto mma_units = [&](const uint32_t (&a)[4][4], const uint32_t (&wd)[B][OPU][WPS], int ob, float (&T)[B][4]) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+#pragma unroll
+            for (int u = 0; u < B; ++u) {
+                if (ob + u < nh) {
+                    // (b0, b1): row g's codes for k = 2q, 2q + 1 and 2q + 8, 2q + 9 of step j
+                    uint32_t b0[OPU], b1[OPU];
+#pragma unroll
+                    for (int h = 0; h < OPU; ++h) {
+                        if (BITS == 4) {           // block j / 2, pairs 2(j % 2) and + 1
+                            b0[h] = dec_u4(wd[u][h][j >> 1], 2 * (j & 1));
+                            b1[h] = dec_u4(wd[u][h][j >> 1], 2 * (j & 1) + 1);
+                        } else if (BITS == 2) {    // the chunk's block, pairs 2j and 2j + 1
+                            b0[h] = dec_t2(wd[u][h][0], 2 * j);
+                            b1[h] = dec_t2(wd[u][h][0], 2 * j + 1);
+                        } else {
+                            const int pc = (j & 1) * 8 + q;
+                            b0[h] = dec_b1(wd[u][h][j >> 1], pc);
+                            b1[h] = dec_b1(wd[u][h][j >> 1], pc + 4);
+                        }
+                    }
+                    if constexpr (SWAP) {
+                        // A = rows g (octet 2u) and g + 8 (octet 2u + 1) of the unit
+                        const uint32_t aw[4] = {b0[0], b0[OPU - 1], b1[0], b1[OPU - 1]};
+                        const uint32_t x0 = a[j >> 1][2 * (j & 1)], x1 = a[j >> 1][2 * (j & 1) + 1];
+                        if (j == 0) mma_bf16_z(T[u], aw, x0, x1);
+                        else mma_bf16(T[u], aw, x0, x1);
+                    } else {
+                        if (j == 0) mma_bf16_z(T[u], a[0], b0[0], b1[0]);
+                        else mma_bf16(T[u], a[j], b0[0], b1[0]);
+                    }
+                }
+            }
+        }
+    };
+    // P6: scale the group sums and add them to the accumulators
+    auto scale_units = [&](const float (&T)[B][4], const float (&tsx)[4], const float4* tab, int ob) {
+#pragma unroll
+        for (int u = 0; u < B; ++u) {
+            if (ob + u < nh) {
+                float* d = acc[ob + u];
+                if constexpr (SWAP) {
+                    // d: (row g, token 2q), (row g, 2q + 1), (row g + 8, 2q), (row g + 8, 2q + 1)
+                    const float4 sc = tab[8 * (ob + u) + g];
+                    d[0] = fmaf(sc.x, T[u][0], d[0]);
+                    d[1] = fmaf(sc.x, T[u][1], d[1]);
+                    d[2] = fmaf(sc.y, T[u][2], d[2]);
+                    d[3] = fmaf(sc.y, T[u][3], d[3]);
+                    if (BITS != 1) {
+                        d[0] = fmaf(-sc.z, tsx[0], d[0]);
+                        d[1] = fmaf(-sc.z, tsx[1], d[1]);
+                        d[2] = fmaf(-sc.w, tsx[0], d[2]);
+                        d[3] = fmaf(-sc.w, tsx[1], d[3]);
+                    }
+                } else {
+                    // d: (token g, row 2q), (g, 2q + 1), (g + 8, 2q), (g + 8, 2q + 1)
+                    const float4 sc = tab[4 * (ob + u) + q];
+                    d[0] = fmaf(sc.x, T[u][0], d[0]);
+                    d[1] = fmaf(sc.y, T[u][1], d[1]);
+                    d[2] = fmaf(sc.x, T[u][2], d[2]);
+                    d[3] = fmaf(sc.y, T[u][3], d[3]);
+                    if (BITS != 1) {
+                        d[0] = fmaf(-sc.z, tsx[0], d[0]);
+                        d[1] = fmaf(-sc.w, tsx[0], d[1]);
+                        d[2] = fmaf(-sc.z, tsx[2], d[2]);
+                        d[3] = fmaf(-sc.w, tsx[2], d[3]);
+                    }
+                }
+            }
+        }
+    };
+    // Release a ring slot; the last warp out queues ring step it + look into it. Once no step is
+    // left to queue, this slot (and every later step's) needs no count.
+    auto release = [&](int it_done, int slot) {
+        __syncwarp();
+        if (lane == 0 && it_done + look < total) {
+            const uint32_t prev = atom_add_acq_rel(&cnt[slot], 1);
+            if ((prev & (kWarps - 1)) == kWarps - 1 && !*abort_flag) {
+                issue(it_done + look, true, true);
+                iss[slot] += 1;
+            }
+        }
+    };
+
     int it = 0;
     int s = 0;                               // ring slot of step it, and its fill parity
     uint32_t ph = 0;
@@ -321,188 +507,30 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = blockIdx.x; t < p.n_tiles; t += gridDim.x) {
         for (int c = 0; c < nst; ++c, ++it) {
             ok = ok && __all_sync(0xffffffffu, mbar_wait(&full[s], ph, abort_flag, p.status));
+            bool released = false;
             if (ok) {
                 const uint8_t* st = ring + s * p.stage_bytes;
-                const uint32_t st_u = smem_u32(st);
-                // this warp's group: fp32 (s, s * c) of every row of its units
-                {
-                    const __half* sh = reinterpret_cast<const __half*>(st + p.s_off) + gi * R;
-                    const __half* zh = reinterpret_cast<const __half*>(st + p.z_off) + gi * R;
-                    auto sc_of = [&](int r, float& sf, float& cf) {
-                        sf = __half2float(sh[r]);
-                        cf = BITS == 4 ? sf * (128.f + __half2float(zh[r])) : BITS == 2 ? 129.f * sf : 0.f;
-                    };
-                    if constexpr (SWAP) {
-                        // entry 8u + g: rows 16u + g and 16u + g + 8 of the warp's units
-#pragma unroll
-                        for (int i0 = 0; i0 < HP; i0 += 32) {
-                            const int i = i0 + lane;
-                            if (i < 8 * nh) {
-                                const int r = 16 * (ob0 + (i >> 3)) + (i & 7);
-                                float s0, c0, s1, c1;
-                                sc_of(r, s0, c0);
-                                sc_of(r + 8, s1, c1);
-                                scr[i] = make_float4(s0, s1, c0, c1);
-                            }
-                        }
-                    } else {
-                        const __half2* sp = reinterpret_cast<const __half2*>(sh) + 4 * ob0;
-                        const __half2* zp = reinterpret_cast<const __half2*>(zh) + 4 * ob0;
-#pragma unroll
-                        for (int i0 = 0; i0 < HP; i0 += 32) {
-                            const int i = i0 + lane;
-                            if (i < 4 * nh) {
-                                const float2 sf = __half22float2(sp[i]);
-                                float c0 = 0.f, c1 = 0.f;
-                                if (BITS == 4) {
-                                    const float2 zf = __half22float2(zp[i]);
-                                    c0 = sf.x * (128.f + zf.x);
-                                    c1 = sf.y * (128.f + zf.y);
-                                } else if (BITS == 2) {
-                                    c0 = 129.f * sf.x;
-                                    c1 = 129.f * sf.y;
-                                }
-                                scr[i] = make_float4(sf.x, sf.y, c0, c1);
-                            }
-                        }
-                    }
-                    // (read back by the other lanes only after the first sub-batch's MMAs)
-                }
-                // X fragments of this warp's four 16-wide K steps (128-byte swizzled rows):
-                // a[j] = the A operand of step j, or with SWAP a[p] = the B operands of steps 2p, 2p + 1
+                build_table(st, scr);         // (read back by the other lanes after the first sub-batch's MMAs)
                 uint32_t a[4][4];
-                if constexpr (SWAP) {
-#pragma unroll
-                    for (int pp = 0; pp < 2; ++pp) {
-                        const int chunk = 4 * pp + (lane >> 3);
-                        ldmatrix_x4(st_u + xoff + static_cast<uint32_t>((chunk ^ tok) << 4), a[pp]);
-                    }
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const int chunk = (j << 1) | xhalf;
-                        ldmatrix_x4(st_u + xoff + static_cast<uint32_t>((chunk ^ (tok & 7)) << 4), a[j]);
-                    }
-                }
-                // group sums of X: tokens g (0) and g + 8 (2), or with SWAP tokens 2q (0) and 2q + 1 (1)
-                float tsx[4] = {0.f, 0.f, 0.f, 0.f};
-                if (BITS != 1) {
-                    if constexpr (SWAP) {
-                        const uint32_t ones[4] = {kBf16One2, kBf16One2, kBf16One2, kBf16One2};
-                        mma_bf16_z(tsx, ones, a[0][0], a[0][1]);
-                        mma_bf16(tsx, ones, a[0][2], a[0][3]);
-                        mma_bf16(tsx, ones, a[1][0], a[1][1]);
-                        mma_bf16(tsx, ones, a[1][2], a[1][3]);
-                    } else {
-                        mma_bf16_z(tsx, a[0], kBf16One2, kBf16One2);
-#pragma unroll
-                        for (int j = 1; j < 4; ++j) mma_bf16(tsx, a[j], kBf16One2, kBf16One2);
-                    }
-                }
-                const uint8_t* wst = st + p.w_off;
+                load_frags(smem_u32(st), a);
+                float tsx[4];
+                group_sums(a, tsx);
 #pragma unroll
                 for (int ob = 0; ob < NH; ob += B) {
-                    // codes of the sub-batch's units for this warp's 64 K
                     uint32_t wd[B][OPU][WPS];
-#pragma unroll
-                    for (int u = 0; u < B; ++u) {
-                        if (ob + u < nh) {
-#pragma unroll
-                            for (int h = 0; h < OPU; ++h) {
-                                const uint8_t* rp = wst + (OPU * (ob0 + ob + u) + h) * kOctStride;
-                                if (BITS == 4) {
-                                    wd[u][h][0] = *reinterpret_cast<const uint32_t*>(rp + wb0);
-                                    wd[u][h][1] = *reinterpret_cast<const uint32_t*>(rp + wb1);
-                                } else if (BITS == 2) {
-                                    wd[u][h][0] = *reinterpret_cast<const uint32_t*>(rp + wb0);
-                                } else {
-                                    const uint2 v = *reinterpret_cast<const uint2*>(rp + wb0);
-                                    wd[u][h][0] = v.x; wd[u][h][1] = v.y;
-                                }
-                            }
-                        }
-                    }
+                    load_codes(st + p.w_off, ob, wd);
                     float T[B][4];
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-#pragma unroll
-                        for (int u = 0; u < B; ++u) {
-                            if (ob + u < nh) {
-                                // (b0, b1): row g's codes for k = 2q, 2q + 1 and 2q + 8, 2q + 9 of step j
-                                uint32_t b0[OPU], b1[OPU];
-#pragma unroll
-                                for (int h = 0; h < OPU; ++h) {
-                                    if (BITS == 4) {           // block j / 2, pairs 2(j % 2) and + 1
-                                        b0[h] = dec_u4(wd[u][h][j >> 1], 2 * (j & 1));
-                                        b1[h] = dec_u4(wd[u][h][j >> 1], 2 * (j & 1) + 1);
-                                    } else if (BITS == 2) {    // the chunk's block, pairs 2j and 2j + 1
-                                        b0[h] = dec_t2(wd[u][h][0], 2 * j);
-                                        b1[h] = dec_t2(wd[u][h][0], 2 * j + 1);
-                                    } else {
-                                        const int pc = (j & 1) * 8 + q;
-                                        b0[h] = dec_b1(wd[u][h][j >> 1], pc);
-                                        b1[h] = dec_b1(wd[u][h][j >> 1], pc + 4);
-                                    }
-                                }
-                                if constexpr (SWAP) {
-                                    // A = rows g (octet 2u) and g + 8 (octet 2u + 1) of the unit
-                                    const uint32_t aw[4] = {b0[0], b0[OPU - 1], b1[0], b1[OPU - 1]};
-                                    const uint32_t x0 = a[j >> 1][2 * (j & 1)], x1 = a[j >> 1][2 * (j & 1) + 1];
-                                    if (j == 0) mma_bf16_z(T[u], aw, x0, x1);
-                                    else mma_bf16(T[u], aw, x0, x1);
-                                } else {
-                                    if (j == 0) mma_bf16_z(T[u], a[0], b0[0], b1[0]);
-                                    else mma_bf16(T[u], a[j], b0[0], b1[0]);
-                                }
-                            }
-                        }
+                    mma_units(a, wd, ob, T);
+                    if (ob + B >= NH) {
+                        release(it, s);       // the last shared-memory read of this slot is done
+                        released = true;
+                    } else if (ob == 0) {
+                        __syncwarp();         // the scale entries above are written
                     }
-                    if (ob == 0) __syncwarp();   // the scale entries above are written
-#pragma unroll
-                    for (int u = 0; u < B; ++u) {
-                        if (ob + u < nh) {
-                            float* d = acc[ob + u];
-                            if constexpr (SWAP) {
-                                // d: (row g, token 2q), (row g, 2q + 1), (row g + 8, 2q), (row g + 8, 2q + 1)
-                                const float4 sc = scr[8 * (ob + u) + g];
-                                d[0] = fmaf(sc.x, T[u][0], d[0]);
-                                d[1] = fmaf(sc.x, T[u][1], d[1]);
-                                d[2] = fmaf(sc.y, T[u][2], d[2]);
-                                d[3] = fmaf(sc.y, T[u][3], d[3]);
-                                if (BITS != 1) {
-                                    d[0] = fmaf(-sc.z, tsx[0], d[0]);
-                                    d[1] = fmaf(-sc.z, tsx[1], d[1]);
-                                    d[2] = fmaf(-sc.w, tsx[0], d[2]);
-                                    d[3] = fmaf(-sc.w, tsx[1], d[3]);
-                                }
-                            } else {
-                                // d: (token g, row 2q), (g, 2q + 1), (g + 8, 2q), (g + 8, 2q + 1)
-                                const float4 sc = scr[4 * (ob + u) + q];
-                                d[0] = fmaf(sc.x, T[u][0], d[0]);
-                                d[1] = fmaf(sc.y, T[u][1], d[1]);
-                                d[2] = fmaf(sc.x, T[u][2], d[2]);
-                                d[3] = fmaf(sc.y, T[u][3], d[3]);
-                                if (BITS != 1) {
-                                    d[0] = fmaf(-sc.z, tsx[0], d[0]);
-                                    d[1] = fmaf(-sc.w, tsx[0], d[1]);
-                                    d[2] = fmaf(-sc.z, tsx[2], d[2]);
-                                    d[3] = fmaf(-sc.w, tsx[2], d[3]);
-                                }
-                            }
-                        }
-                    }
+                    scale_units(T, tsx, scr, ob);
                 }
             }
-            __syncwarp();
-            // Release the slot; the last warp out queues ring step it + look = it + S into it. Once
-            // no step is left to queue, this slot (and every later step's) needs no count.
-            if (lane == 0 && it + look < total) {
-                const uint32_t prev = atom_add_acq_rel(&cnt[s], 1);
-                if ((prev & (kWarps - 1)) == kWarps - 1 && !*abort_flag) {
-                    issue(it + look, true, true);
-                    iss[s] += 1;
-                }
-            }
+            if (!released) release(it, s);
             if (++s == S) {
                 s = 0;
                 ph ^= 1u;
