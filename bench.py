@@ -39,14 +39,27 @@ DEFAULT_WORKLOAD = "klein_step_chain_1024sq_ternary_g128"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
-def kernel_source_hash():
-    """sha256 over the CUDA sources and the ABI header: identifies the kernels a capture measured."""
+# The sources each kernel is built from (besides the headers every kernel includes): a capture
+# stays valid while these are unchanged.
+KERNEL_SOURCES = {"lowbit_gemm_kernel": ("gemm_sm100.cu",),
+                  "lowbit_smallm_kernel": ("smallm_kernel.cuh", "smallm_host.cu", "smallm_b1.cu", "smallm_b2.cu",
+                                           "smallm_b4.cu")}
+SHARED_SOURCES = ("sm100_ptx.cuh", "lowbit_internal.h")
+
+
+def kernel_source_hash(kernel=None):
+    """sha256 over the sources a kernel is built from (all CUDA sources and the ABI header when
+    `kernel` is None): identifies the code a capture measured."""
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "bit_weight_only_w2_b200", "csrc")
     inc = os.path.join(ROOT, "include")
-    files = sorted(os.path.join(csrc, f) for f in os.listdir(csrc) if f.endswith((".cu", ".cuh", ".h")))
-    files += sorted(os.path.join(inc, f) for f in os.listdir(inc) if f.endswith(".h"))
+    if kernel is None:
+        files = sorted(os.path.join(csrc, f) for f in os.listdir(csrc) if f.endswith((".cu", ".cuh", ".h")))
+        files += sorted(os.path.join(inc, f) for f in os.listdir(inc) if f.endswith(".h"))
+    else:
+        files = [os.path.join(csrc, f) for f in (*KERNEL_SOURCES[kernel], *SHARED_SOURCES)]
+        files += [os.path.join(inc, "lowbit.h")]
     for f in files:
         h.update(os.path.basename(f).encode())
         with open(f, "rb") as fh:
@@ -56,13 +69,13 @@ def kernel_source_hash():
 
 def measured_traffic(key):
     """DRAM bytes per launch from the committed ncu summary for this workload, or None if there is
-    none or the kernels have changed since it was captured."""
+    none or the captured kernel's sources have changed since."""
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             entry = json.load(f).get(key)
     except Exception:
         return None
-    if not entry or entry.get("source_sha256") != kernel_source_hash():
+    if not entry or entry.get("source_sha256") != kernel_source_hash(entry.get("kernel")):
         return None
     return entry.get("dram_bytes_per_launch")
 

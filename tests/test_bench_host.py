@@ -140,3 +140,23 @@ def test_world_must_match_gpus():
     with pytest.raises(SystemExit):
         bench.check_world(4, 2)
 
+
+
+def test_traffic_follows_only_its_own_kernels_sources(tmp_path, monkeypatch):
+    """A capture of one kernel stays valid when only another kernel's sources change."""
+    csrc = tmp_path / "bit_weight_only_w2_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    for f in (*bench.KERNEL_SOURCES["lowbit_gemm_kernel"], *bench.KERNEL_SOURCES["lowbit_smallm_kernel"],
+              *bench.SHARED_SOURCES):
+        (csrc / f).write_text(f"// {f}\n")
+    (tmp_path / "include").mkdir()
+    (tmp_path / "include" / "lowbit.h").write_text("/* header */\n")
+    (tmp_path / "profiles").mkdir()
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    h = bench.kernel_source_hash("lowbit_gemm_kernel")
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(
+        {"w": {"dram_bytes_per_launch": 7.0, "source_sha256": h, "kernel": "lowbit_gemm_kernel"}}))
+    (csrc / "smallm_kernel.cuh").write_text("// changed\n")
+    assert bench.measured_traffic("w") == 7.0
+    (csrc / "sm100_ptx.cuh").write_text("// changed\n")          # shared by every kernel
+    assert bench.measured_traffic("w") is None
