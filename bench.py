@@ -160,6 +160,61 @@ def measure_shapes(items, copies, lb, torch, device, stream, cap_stream, samples
 
 CONFIGS = ("tiny_ternary_g64", "qkv_512sq_ternary_g128", "mlp_1024sq_binary_g128", "te_m512_uint4_g64",
            "te_m16_uint4_g64", "klein_linears_m1_ternary_g128")
+# Whole-step workloads measured beside them: the transformer step with separate Q/K/V and
+# add-Q/K/V projections (100 linears) and the text encoder's 4-layer MLP chain at 512 and 16 tokens.
+STEP_CONFIGS = ("klein_step_linears100_1024sq_ternary_g128", "te_mlp4_m512_uint4_g64", "te_mlp4_m16_uint4_g64")
+
+
+def capture_steps(lb, torch, desc_sets, device, stream, cap_stream):
+    """One CUDA graph per weight copy, each holding one lowbit_gemm_batch over the step's linears
+    (replaying a graph measures the GPU, not the host's per-call submission cost)."""
+    lb.gemm_batch(desc_sets[0], device)   # allocates the shared workspace before capture
+    torch.cuda.synchronize(device)
+    graphs = []
+    cap_stream.wait_stream(stream)
+    with torch.cuda.stream(cap_stream):
+        for descs in desc_sets:
+            gph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gph, stream=cap_stream):
+                lb.gemm_batch(descs, device)
+            graphs.append(gph)
+    stream.wait_stream(cap_stream)
+    torch.cuda.synchronize(device)
+    return graphs
+
+
+def measure_step_config(name, lb, torch, device, stream, cap_stream, peaks, l2_bytes, steps=10, samples=5):
+    """Step time of a whole workload run as one lowbit_gemm_batch per step (graph-replayed, weight
+    copies rotated below twice L2): the median over `samples` samples of `steps` steps each."""
+    specs = synth.WORKLOADS[name]
+    flops, nbytes = step_flops(specs), step_bytes(specs)
+    copies = rotation_copies(nbytes, weight_bytes(specs), l2_bytes)
+    items, desc_sets = setup(specs, device, lb, torch, pinned=False, copies=copies)   # items own the buffers
+    graphs = capture_steps(lb, torch, desc_sets, device, stream, cap_stream)
+    n = max(steps, copies)
+    for i in range(max(3, copies)):
+        graphs[i % copies].replay()
+    torch.cuda.synchronize(device)
+    ts = []
+    for _ in range(samples):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(n):
+            graphs[i % copies].replay()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        ts.append(e0.elapsed_time(e1) / n)
+    ms = statistics.median(ts)
+    hbm = is_hbm_bound(flops, nbytes, peaks)
+    out = {"linears_per_step": len(specs), "ms_per_step": ms, "tflops": flops / (ms * 1e-3) / 1e12,
+           "gbs": nbytes / (ms * 1e-3) / 1e9, "bound": "hbm" if hbm else "tensor",
+           "weight_copies_rotated": copies, "steps_per_sample": n}
+    if hbm:
+        out["frac_of_hbm"] = out["gbs"] / peaks.get("hbm_gbs")
+    else:
+        out["frac_of_burst"] = out["tflops"] / peaks.get("bf16_tflops")
+    del graphs, desc_sets, items
+    return out
 
 
 def measure_configs(lb, torch, device, stream, cap_stream, peaks, l2_bytes):
@@ -189,6 +244,12 @@ def measure_configs(lb, torch, device, stream, cap_stream, peaks, l2_bytes):
         del items
         torch.cuda.synchronize(device)
         torch.cuda.empty_cache()
+    for name in STEP_CONFIGS:
+        out[name] = {"step": measure_step_config(name, lb, torch, device, stream, cap_stream, peaks, l2_bytes)}
+        torch.cuda.synchronize(device)
+        torch.cuda.empty_cache()
+    if lb.device_status() != 0:
+        raise RuntimeError("kernel timeout reported while measuring the reference configurations")
     return out
 
 
@@ -439,21 +500,9 @@ def run_lowbit(args, specs, workload):
         return max_over_ranks(v, world, device)
 
     # Each step is one lowbit_gemm_batch over the workload's linears, captured once per weight
-    # copy as a CUDA graph and replayed, so the timed region measures the GPU rather than the
-    # host's per-call submission cost (the end-to-end number below calls the API directly).
-    lb.gemm_batch(desc_sets[0], device)   # allocates the shared workspace before capture
-    torch.cuda.synchronize(device)
-    graphs = []
+    # copy as a CUDA graph and replayed (the end-to-end number below calls the API directly).
     cap_stream = torch.cuda.Stream(device)
-    cap_stream.wait_stream(stream)
-    with torch.cuda.stream(cap_stream):
-        for c in range(copies):
-            gph = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(gph, stream=cap_stream):
-                lb.gemm_batch(desc_sets[c], device)
-            graphs.append(gph)
-    stream.wait_stream(cap_stream)
-    torch.cuda.synchronize(device)
+    graphs = capture_steps(lb, torch, desc_sets[:copies], device, stream, cap_stream)
     step_idx = [0]
 
     def one_step():
