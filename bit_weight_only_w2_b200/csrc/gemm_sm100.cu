@@ -63,11 +63,16 @@ constexpr int kBlockK = 128;        // K per pipeline stage
 constexpr int kNumCtrlWarps = 2;    // warp 0: TMA producer, warp 1: MMA issuer + TMEM owner
 constexpr int kSmemLimit = 232448;  // 227 KB opt-in dynamic shared memory per block
 
-template <int BITS, int GS, int BT>
+// PAIR: a tile of 256 weight rows x BT tokens computed by a CTA pair on cta_group::2 MMAs. Each
+// CTA decodes its 128 weight rows into its own tensor memory and loads half of the X tile (BT/2
+// tokens); the even CTA issues the MMAs, which read both halves of X, so every X element read
+// into shared memory serves 256 weight rows instead of 128.
+template <int BITS, int GS, int BT, bool PAIR = false>
 struct Cfg {
     static_assert(BITS == 1 || BITS == 2 || BITS == 4, "bits");
     static_assert(GS == 64 || GS == 128, "group size");
     static_assert(BT % 16 == 0 && BT >= 16 && BT <= 256, "MMA N");
+    static_assert(!PAIR || BT == 256, "pair tiles are 256 x 256");
     static constexpr int kCtasPerSm = (BT <= 64) ? 2 : 1;
     // Epilogue: warps e and e+4 cover the same 32 weight rows (TMEM lane quarter = warp % 4),
     // each half of the tile's token columns when there are 8.
@@ -90,7 +95,8 @@ struct Cfg {
 
     static constexpr int kWordsPerRow = kBlockK * BITS / 32;        // 4 / 8 / 16
     static constexpr int kWRowBytes = kWordsPerRow * 4;             // 16 / 32 / 64
-    static constexpr int kXHalfBytes = BT * 128;                    // 64 fp16 per row
+    static constexpr int kXRows = PAIR ? BT / 2 : BT;               // token rows of X in this CTA
+    static constexpr int kXHalfBytes = kXRows * 128;                // 64 fp16 per row
     static constexpr int kXBytes = 2 * kXHalfBytes;
     static constexpr int kWBytes = kBlockN * kWRowBytes;
     static constexpr int kGroupsPerStage = kBlockK / GS;            // 1 or 2
@@ -125,7 +131,7 @@ struct Cfg {
     // split-K partial tile (fp32 [128][BT], rows of 16-byte chunks XOR-swizzled) reuses the X ring
     static_assert(BT * kBlockN * 4 <= kXStages * kXStageBytes, "split-K partial buffer");
     static constexpr int kPartSwizzle = (BT / 4 >= 8) ? 7 : (BT / 4 - 1);
-    static constexpr uint32_t kIdesc = idesc_f16_f32(kBlockN, BT);
+    static constexpr uint32_t kIdesc = idesc_f16_f32(PAIR ? 2 * kBlockN : kBlockN, BT);
 };
 
 struct KernelParams {
@@ -205,12 +211,12 @@ __device__ __forceinline__ void decode_word_b4(uint32_t v, uint16_t s, float cz,
 // ---------------------------------------------------------------------------------------------
 // The kernel
 // ---------------------------------------------------------------------------------------------
-template <int BITS, int GS, int BT>
-__global__ void __launch_bounds__(Cfg<BITS, GS, BT>::kThreads, Cfg<BITS, GS, BT>::kCtasPerSm)
+template <int BITS, int GS, int BT, bool PAIR>
+__global__ void __launch_bounds__(Cfg<BITS, GS, BT, PAIR>::kThreads, Cfg<BITS, GS, BT, PAIR>::kCtasPerSm)
     lowbit_gemm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w,
                        const __grid_constant__ CUtensorMap map_s, const __grid_constant__ CUtensorMap map_z,
                        const KernelParams p) {
-    using C = Cfg<BITS, GS, BT>;
+    using C = Cfg<BITS, GS, BT, PAIR>;
     constexpr int SX = C::kXStages;
     constexpr int SW = C::kWStages;
     constexpr int NA = C::kNumA;
@@ -233,6 +239,14 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT>::kThreads, Cfg<BITS, GS, BT>
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    // Pair mode: the CTA of cluster rank 0 issues the MMAs. The other CTA's X copies complete on
+    // the issuer's X barrier, its dequant and epilogue warps arrive on the issuer's A-ready and
+    // accumulator-free barriers, and the issuer's commits arrive on the empty / ready barriers of
+    // both CTAs (same offsets).
+    const uint32_t pair_rank = PAIR ? cluster_ctarank() : 0u;
+    const bool issuer = pair_rank == 0;
+    constexpr int kPairCtas = PAIR ? 2 : 1;
+    auto on_issuer = [&](uint64_t* bar) { return map_shared_rank(smem_u32(bar), 0u); };
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < SX; ++i) {
@@ -244,12 +258,12 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT>::kThreads, Cfg<BITS, GS, BT>
             mbar_init(&wempty[i], C::kNumDqWarps);
         }
         for (int i = 0; i < NA; ++i) {
-            mbar_init(&afull[i], C::kNumDqWarps);
+            mbar_init(&afull[i], kPairCtas * C::kNumDqWarps);
             mbar_init(&aempty[i], 1);
         }
         for (int i = 0; i < NACC; ++i) {
             mbar_init(&accfull[i], 1);
-            mbar_init(&accempty[i], C::kNumEpiWarps);
+            mbar_init(&accempty[i], kPairCtas * C::kNumEpiWarps);
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -262,11 +276,12 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT>::kThreads, Cfg<BITS, GS, BT>
         if (BITS == 4) tma_prefetch_desc(&map_z);
     }
     if (warp == 1) {
-        tmem_alloc(tmem_holder, C::kTmemCols);
-        tmem_relinquish();
+        tmem_alloc<PAIR>(tmem_holder, C::kTmemCols);
+        tmem_relinquish<PAIR>();
     }
     tc_fence_before();
     __syncthreads();
+    if (PAIR) cluster_sync_all();   // both CTAs' barriers are initialised before either uses the other's
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
 
@@ -278,9 +293,14 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT>::kThreads, Cfg<BITS, GS, BT>
     const int kb_begin = split ? static_cast<int>(blockIdx.z) * p.kb_per_split : 0;
     const int kb_end = split ? min(p.num_kb, kb_begin + p.kb_per_split) : p.num_kb;
     const int nkb = kb_end - kb_begin;
-    const int tile_step = split ? p.num_tiles : static_cast<int>(gridDim.x);
-    const int my_tiles =
-        static_cast<int>(blockIdx.x) < p.num_tiles ? (p.num_tiles - 1 - static_cast<int>(blockIdx.x)) / tile_step + 1 : 0;
+    // first tile and tile stride of this CTA (a pair's two CTAs, adjacent along x, share both)
+    const int tile0 = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+    const int tile_step = split ? p.num_tiles : static_cast<int>(PAIR ? gridDim.x >> 1 : gridDim.x);
+    const int my_tiles = tile0 < p.num_tiles ? (p.num_tiles - 1 - tile0) / tile_step + 1 : 0;
+    // first weight row of this CTA in tile t: pair tiles cover 2 * p.rows rows, this CTA's half
+    // starting at pair_rank * p.rows
+    const int n_stride = PAIR ? 2 * p.rows : p.rows;
+    const int n_off = PAIR ? static_cast<int>(pair_rank) * p.rows : 0;
     unsigned* status = &g_device_status;
 
     if (warp == 0) {
@@ -288,10 +308,10 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT>::kThreads, Cfg<BITS, GS, BT>
         if (lane == 0) {
             const uint32_t total = static_cast<uint32_t>(my_tiles * nkb);
             auto coords = [&](uint32_t it, int& m0, int& n0, int& kb) {
-                const int tile = static_cast<int>(blockIdx.x) + static_cast<int>(it / nkb) * tile_step;
+                const int tile = tile0 + static_cast<int>(it / nkb) * tile_step;
                 kb = kb_begin + static_cast<int>(it % nkb);
                 m0 = (tile / p.n_tiles) * BT;
-                n0 = (tile % p.n_tiles) * p.rows;
+                n0 = (tile % p.n_tiles) * n_stride + n_off;
             };
             auto issue_w = [&](uint32_t it) {
                 int m0, n0, kb;
@@ -308,9 +328,16 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT>::kThreads, Cfg<BITS, GS, BT>
                 coords(it, m0, n0, kb);
                 const uint32_t s = it % SX;
                 uint8_t* st = smem + s * C::kXStageBytes;
-                mbar_arrive_expect_tx(&xfull[s], C::kXBytes);
-                // box (64 k, BT tokens, 2 halves) = both 128-byte-swizzled K halves in one request
-                tma_load_3d(&map_x, &xfull[s], st, 0, m0, kb * 2);
+                // box (64 k, kXRows tokens, 2 halves) = both 128-byte-swizzled K halves in one request
+                if (!PAIR) {
+                    mbar_arrive_expect_tx(&xfull[s], C::kXBytes);
+                    tma_load_3d(&map_x, &xfull[s], st, 0, m0, kb * 2);
+                } else {
+                    // both halves complete on the issuer's barrier, which expects both
+                    if (issuer) mbar_arrive_expect_tx(&xfull[s], 2 * C::kXBytes);
+                    tma_load_3d_pair(&map_x, on_issuer(&xfull[s]), st, 0, m0 + static_cast<int>(pair_rank) * C::kXRows,
+                                     kb * 2);
+                }
             };
             // The packed weights and scales are not written by the kernel just before this one
             // (the X conversion, which itself starts only once everything earlier in the stream
@@ -347,10 +374,18 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT>::kThreads, Cfg<BITS, GS, BT>
                 }
             }
             if (!ok) {
-                // Drain: wait (bounded) for the copies still in flight before the CTA exits.
-                for (uint32_t j = (itx > static_cast<uint32_t>(SX) ? itx - SX : 0u); j < itx; ++j) {
+                // Drain: wait (bounded) for the copies still in flight before the CTA exits. The
+                // second CTA of a pair cannot wait on the issuer's barrier its X copies count on:
+                // it gives them a fixed time instead (both CTAs meet again before either exits).
+                if (PAIR && !issuer) {
                     const long long t0 = clock64();
-                    while (!mbar_try_wait(&xfull[j % SX], (j / SX) & 1u) && clock64() - t0 < kWaitLimitCycles) {
+                    while (clock64() - t0 < kWaitLimitCycles / 64) {
+                    }
+                } else {
+                    for (uint32_t j = (itx > static_cast<uint32_t>(SX) ? itx - SX : 0u); j < itx; ++j) {
+                        const long long t0 = clock64();
+                        while (!mbar_try_wait(&xfull[j % SX], (j / SX) & 1u) && clock64() - t0 < kWaitLimitCycles) {
+                        }
                     }
                 }
                 for (uint32_t j = (itw > static_cast<uint32_t>(SW) ? itw - SW : 0u); j < itw; ++j) {
@@ -362,7 +397,7 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT>::kThreads, Cfg<BITS, GS, BT>
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA issuer
-        if (lane == 0) {
+        if (lane == 0 && issuer) {
             uint32_t it = 0, ait = 0, tcount = 0;
             bool ok = true;
             bool issued = false;
@@ -386,18 +421,32 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT>::kThreads, Cfg<BITS, GS, BT>
                         const uint32_t a_tmem = tmem_base + C::kACol0 + a * 64 + kk * 8;
                         const uint64_t bdesc =
                             smem_desc_k_sw128(xs + (kk >> 2) * C::kXHalfBytes + (kk & 3) * 32);
-                        mma_f16_ts(d_tmem, a_tmem, bdesc, C::kIdesc, (kb > kb_begin || kk > 0) ? 1u : 0u);
+                        if (PAIR)
+                            mma_f16_ts_pair(d_tmem, a_tmem, bdesc, C::kIdesc, (kb > kb_begin || kk > 0) ? 1u : 0u);
+                        else
+                            mma_f16_ts(d_tmem, a_tmem, bdesc, C::kIdesc, (kb > kb_begin || kk > 0) ? 1u : 0u);
                     }
                     issued = true;
-                    mma_commit(&xempty[s]);
-                    mma_commit(&aempty[a]);
+                    if (PAIR) {
+                        mma_commit_pair_mc(&xempty[s], 0x3);
+                        mma_commit_pair_mc(&aempty[a], 0x3);
+                    } else {
+                        mma_commit(&xempty[s]);
+                        mma_commit(&aempty[a]);
+                    }
                 }
                 if (!ok) break;
-                mma_commit(&accfull[b]);
+                if (PAIR)
+                    mma_commit_pair_mc(&accfull[b], 0x3);
+                else
+                    mma_commit(&accfull[b]);
             }
             if (!ok && issued) {
                 // Drain: make sure no MMA is still writing tensor memory before it is freed.
-                mma_commit(drain);
+                if (PAIR)
+                    mma_commit_pair(drain);
+                else
+                    mma_commit(drain);
                 const long long t0 = clock64();
                 while (!mbar_try_wait(drain, 0) && clock64() - t0 < kWaitLimitCycles) {
                 }
@@ -489,7 +538,12 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT>::kThreads, Cfg<BITS, GS, BT>
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&afull[a]);
+                if (lane == 0) {
+                    if (PAIR && !issuer)
+                        mbar_arrive_remote(on_issuer(&afull[a]));
+                    else
+                        mbar_arrive(&afull[a]);
+                }
             }
         }
     } else {
@@ -506,10 +560,10 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT>::kThreads, Cfg<BITS, GS, BT>
         uint32_t tcount = 0;
         constexpr int kChunks = C::kEpiCols / kChunk;
         for (int t = 0; t < my_tiles; ++t, ++tcount) {
-            const int tile = static_cast<int>(blockIdx.x) + t * tile_step;
+            const int tile = tile0 + t * tile_step;
             const uint32_t b = tcount % NACC, acc_ph = (tcount / NACC) & 1u;
             const int m0 = (tile / p.n_tiles) * BT + col0;   // first token of this thread's columns
-            const int n = (tile % p.n_tiles) * p.rows + row;
+            const int n = (tile % p.n_tiles) * n_stride + n_off + row;
             // Lane j of the warp holds the row factor of token m0 + c0 + j of every chunk c0,
             // requested before waiting for the accumulator so the loads overlap the MMAs.
             float mul[kChunks];
@@ -545,7 +599,12 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT>::kThreads, Cfg<BITS, GS, BT>
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&accempty[b]);
+                if (lane == 0) {
+                    if (PAIR && !issuer)
+                        mbar_arrive_remote(on_issuer(&accempty[b]));
+                    else
+                        mbar_arrive(&accempty[b]);
+                }
                 // Lanes 2i and 2i+1 hold rows n and n+1: one shuffle turns each lane's
                 // (token m, token m+1) pair into a 4-byte (row n, row n+1) store at one token.
                 const bool even = (lane & 1) == 0;
@@ -665,9 +724,12 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT>::kThreads, Cfg<BITS, GS, BT>
 
     tc_fence_before();
     __syncthreads();
+    // a pair's tensor memory is freed by both CTAs together, once neither uses it (and no
+    // remote arrival or copy of one CTA targets the other after it has exited)
+    if (PAIR) cluster_sync_all();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, C::kTmemCols);
+        tmem_dealloc<PAIR>(tmem_base, C::kTmemCols);
     }
 }
 
@@ -921,10 +983,12 @@ bool make_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, int elem_bytes, co
     return encode_cached(map, dtype, 2, base, dims, strides, box, swz);
 }
 
-int cluster_capacity(const void* kernel, int ks, int threads, int smem_bytes) {
+int cluster_capacity(const void* kernel, int ks, int threads, int smem_bytes, bool along_x = false) {
     struct Entry {
         const void* fn;
-        int dev, ks, cap;
+        int dev, ks;
+        bool x;
+        int cap;
     };
     static Entry cache[64];
     static int used = 0;
@@ -934,16 +998,17 @@ int cluster_capacity(const void* kernel, int ks, int threads, int smem_bytes) {
     {
         std::lock_guard<std::mutex> lock(mu);
         for (int i = 0; i < used; ++i)
-            if (cache[i].fn == kernel && cache[i].dev == dev && cache[i].ks == ks) return cache[i].cap;
+            if (cache[i].fn == kernel && cache[i].dev == dev && cache[i].ks == ks && cache[i].x == along_x)
+                return cache[i].cap;
     }
     int n = 0;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.x = along_x ? ks : 1;
     attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = ks;
-    cfg.gridDim = dim3(1, 1, ks);
+    attr[0].val.clusterDim.z = along_x ? 1 : ks;
+    cfg.gridDim = along_x ? dim3(ks, 1, 1) : dim3(1, 1, ks);
     cfg.blockDim = dim3(threads, 1, 1);
     cfg.dynamicSmemBytes = smem_bytes;
     cfg.attrs = attr;
@@ -953,7 +1018,7 @@ int cluster_capacity(const void* kernel, int ks, int threads, int smem_bytes) {
         n = num_sms() / ks;
     }
     std::lock_guard<std::mutex> lock(mu);
-    if (used < 64) cache[used++] = Entry{kernel, dev, ks, n};
+    if (used < 64) cache[used++] = Entry{kernel, dev, ks, along_x, n};
     return n;
 }
 
@@ -976,10 +1041,13 @@ int num_sms() {
 
 namespace {
 
-template <int BITS, int GS, int BT>
+// rows: weight rows per CTA tile (0 = automatic: 128, or a CTA pair's 256 where that applies).
+template <int BITS, int GS, int BT, bool PAIR = false>
 lowbit_status launch(const GemmProblem& g, int rows, int ksplit_request, cudaStream_t stream, bool convert_x) {
-    using C = Cfg<BITS, GS, BT>;
-    auto kernel = lowbit_gemm_kernel<BITS, GS, BT>;
+    using C = Cfg<BITS, GS, BT, PAIR>;
+    auto kernel = lowbit_gemm_kernel<BITS, GS, BT, PAIR>;
+    const bool auto_rows = rows == 0;
+    if (auto_rows || PAIR) rows = kBlockN;
     // the shared-memory opt-in is per device: one bit per device that has it
     static std::atomic<uint64_t> attr_devices{0};
     int dev = 0;
@@ -998,7 +1066,7 @@ lowbit_status launch(const GemmProblem& g, int rows, int ksplit_request, cudaStr
     const WorkspaceLayout ws = workspace_layout(g.M, g.K);
     void* xh = g.workspace;
     float* rowmul = reinterpret_cast<float*>(static_cast<uint8_t*>(g.workspace) + ws.rowmul_offset);
-    bool ok = make_map_x3d(&mx, xh, M, K, BT);
+    bool ok = make_map_x3d(&mx, xh, M, K, C::kXRows);
     ok = ok && make_map_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, g.Wp, uint64_t(K) * BITS / 32, N,
                            uint64_t(K) * BITS / 8, C::kWordsPerRow, rows, wswz);
     ok = ok && make_map_2d(&ms, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, g.scales, N, K / GS, uint64_t(N) * 2, kBlockN,
@@ -1018,11 +1086,11 @@ lowbit_status launch(const GemmProblem& g, int rows, int ksplit_request, cudaStr
     p.rows = rows;
     p.wtx_bytes = static_cast<uint32_t>(C::kWTxFixed + rows * C::kWRowBytes);
     p.m_tiles = (M + BT - 1) / BT;
-    p.n_tiles = (N + rows - 1) / rows;
+    p.n_tiles = PAIR ? N / (2 * rows) : (N + rows - 1) / rows;
     p.num_tiles = p.m_tiles * p.n_tiles;
     p.Y = static_cast<__nv_bfloat16*>(g.Y);
     p.rowmul = rowmul;
-    int ksplit = ksplit_request;
+    int ksplit = PAIR ? 1 : ksplit_request;
     if (ksplit < 0) {
         // Automatic: the largest split that leaves every rank at least 24 k-blocks (3072 of K)
         // and keeps all clusters resident at once (the split grid is not persistent, so a
@@ -1040,6 +1108,11 @@ lowbit_status launch(const GemmProblem& g, int rows, int ksplit_request, cudaStr
     }
     if (ksplit < 1) ksplit = 1;
     if (ksplit > 8) ksplit = 8;
+    // An unsplit grid of 256-token tiles over a multiple of 256 weight rows runs on CTA pairs.
+    if constexpr (BT == 256 && !PAIR) {
+        if (auto_rows && ksplit == 1 && N % (2 * kBlockN) == 0)
+            return launch<BITS, GS, BT, true>(g, 0, 1, stream, convert_x);
+    }
     if (ksplit > p.num_kb) ksplit = p.num_kb;
     int kbps = (p.num_kb + ksplit - 1) / ksplit;
     ksplit = (p.num_kb + kbps - 1) / kbps;     // every rank gets at least one k-block
@@ -1056,7 +1129,18 @@ lowbit_status launch(const GemmProblem& g, int rows, int ksplit_request, cudaStr
     attrs[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attrs[na].val.programmaticStreamSerializationAllowed = 1;
     ++na;
-    if (ksplit > 1) {
+    if (PAIR) {
+        // persistent grid of CTA pairs, the two CTAs of a pair adjacent along x (clusters of 2)
+        int pairs = cluster_capacity(reinterpret_cast<const void*>(kernel), 2, C::kThreads, C::kSmemBytes, true);
+        if (pairs > num_sms() / 2) pairs = num_sms() / 2;
+        if (pairs < 1) pairs = 1;
+        cfg.gridDim = dim3(2 * (p.num_tiles < pairs ? p.num_tiles : pairs), 1, 1);
+        attrs[na].id = cudaLaunchAttributeClusterDimension;
+        attrs[na].val.clusterDim.x = 2;
+        attrs[na].val.clusterDim.y = 1;
+        attrs[na].val.clusterDim.z = 1;
+        ++na;
+    } else if (ksplit > 1) {
         cfg.gridDim = dim3(p.num_tiles, 1, ksplit);
         attrs[na].id = cudaLaunchAttributeClusterDimension;
         attrs[na].val.clusterDim.x = 1;
@@ -1095,7 +1179,9 @@ lowbit_status launch_bits_gs(const GemmProblem& g, int bt, int rows, int ksplit,
         case 32: return launch<BITS, GS, 32>(g, rows, ksplit, s, cx);
         case 64: return launch<BITS, GS, 64>(g, rows, ksplit, s, cx);
         case 128: return launch<BITS, GS, 128>(g, rows, ksplit, s, cx);
-        case 256: return launch<BITS, GS, 256>(g, rows, ksplit, s, cx);
+        case 256:
+            if (rows == 2 * kBlockN) return launch<BITS, GS, 256, true>(g, 0, 1, s, cx);
+            return launch<BITS, GS, 256>(g, rows, ksplit, s, cx);
         default: return LOWBIT_ERR_UNSUPPORTED;
     }
 }
@@ -1144,7 +1230,11 @@ lowbit_status gemm_launch(const GemmProblem& g, int force_bt, int force_rows, in
         }
     }
     if (!ksplit) ksplit = 1;
-    if (rows < 8 || rows > kBlockN || rows % 8) return LOWBIT_ERR_UNSUPPORTED;   // (ksplit -1: automatic)
+    // 256 rows: one tile per CTA pair (256-token tiles, N a multiple of 256, no K split)
+    const bool pair_rows = force_rows == 2 * kBlockN;
+    if (pair_rows && (bt != 256 || g.N % (2 * kBlockN) != 0 || ksplit > 1)) return LOWBIT_ERR_UNSUPPORTED;
+    if (!pair_rows && (rows < 8 || rows > kBlockN || rows % 8)) return LOWBIT_ERR_UNSUPPORTED;   // (ksplit -1: automatic)
+    if (!force_rows && rows == kBlockN) rows = 0;   // automatic: the launch may use CTA pairs
     switch (g.bits * 1000 + g.group_size) {
         case 1064: return launch_bits_gs<1, 64>(g, bt, rows, ksplit, stream, convert_x);
         case 1128: return launch_bits_gs<1, 128>(g, bt, rows, ksplit, stream, convert_x);

@@ -183,7 +183,8 @@ LOWBIT_API lowbit_status lowbit_gemm_ex(int64_t M, int64_t N, int64_t K, int bit
     if ((tile_tokens == 1 && M > 16) || (tile_tokens == 8 && M > 8)) return LOWBIT_ERR_UNSUPPORTED;
     if (tile_tokens == 8 && tile_rows % 16 != 0) return LOWBIT_ERR_UNSUPPORTED;
     if (ksplit < 0 || ksplit > 8) return LOWBIT_ERR_UNSUPPORTED;
-    if (tile_rows < 0 || tile_rows > 128 || tile_rows % 8 != 0) return LOWBIT_ERR_UNSUPPORTED;
+    if (tile_rows < 0 || tile_rows % 8 != 0) return LOWBIT_ERR_UNSUPPORTED;
+    if (tile_rows > 128 && !(tile_rows == 256 && (tile_tokens == 0 || tile_tokens == 256))) return LOWBIT_ERR_UNSUPPORTED;
     if ((st = check_device()) != LOWBIT_OK) return st;
     return gemm_launch(g, tile_tokens, tile_rows, ksplit, static_cast<cudaStream_t>(stream));
 }

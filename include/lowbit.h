@@ -134,7 +134,10 @@ lowbit_status lowbit_gemm(int64_t M, int64_t N, int64_t K, int bits, int group_s
  *                scale, so its results are exact only for |x| below about 2^114; the
  *                tensor-memory kernel (M > 16, or tile_tokens >= 16) covers the full bf16 range
  *   tile_rows    weight rows per CTA tile: a multiple of 8 up to 128 (128 unless the shape is
- *                small; fewer rows give more CTAs, each streaming the whole K)
+ *                small; fewer rows give more CTAs, each streaming the whole K), or 256: one
+ *                256 x 256 tile per pair of CTAs on paired tensor-core MMAs (tile_tokens 0 or
+ *                256, 256-token tiles, N % 256 == 0, no K split; chosen automatically for
+ *                unsplit 256-token tiles when N % 256 == 0)
  *   ksplit       number of K slices summed across a thread-block cluster, 1..8 (1 = no split;
  *                the small-M kernel cuts K into slices of whole 512-wide steps, so a request
  *                may be served with fewer slices)

@@ -94,6 +94,13 @@ def test_gemm_ex_rejects_bad_tile(lib):
     assert st == 3
     st = lib.lowbit_gemm_ex(16, 128, 256, 2, 128, A, A, A, None, A, A, WS, 16, 136, 0, None)  # rows > 128
     assert st == 3
+    # 256 rows = a tile per CTA pair: only with 256-token tiles (or the automatic width)
+    st = lib.lowbit_gemm_ex(16, 256, 256, 2, 128, A, A, A, None, A, A, WS, 16, 256, 0, None)
+    assert st == 3
+    st = lib.lowbit_gemm_ex(16, 256, 256, 2, 128, A, A, A, None, A, A, WS, 1, 256, 0, None)
+    assert st == 3
+    st = lib.lowbit_gemm_ex(16, 512, 256, 2, 128, A, A, A, None, A, A, WS, 0, 264, 0, None)
+    assert st == 3
     # the small-M kernel (tile_tokens = 1) serves at most 16 tokens
     st = lib.lowbit_gemm_ex(17, 128, 256, 2, 128, A, A, A, None, A, A, WS, 1, 0, 0, None)
     assert st == 3
