@@ -128,9 +128,17 @@ struct Cfg {
     static constexpr int kSmemFloor = (kCtasPerSm == 2) ? 80 * 1024 : 150 * 1024;
     static constexpr int kSmemBytes = kSmemNeeded > kSmemFloor ? kSmemNeeded : kSmemFloor;
     static_assert(kSmemBytes <= kSmemLimit, "shared memory");
-    // split-K partial tile (fp32 [128][BT], rows of 16-byte chunks XOR-swizzled) reuses the X ring
-    static_assert(BT * kBlockN * 4 <= kXStages * kXStageBytes, "split-K partial buffer");
-    static constexpr int kPartSwizzle = (BT / 4 >= 8) ? 7 : (BT / 4 - 1);
+    // split-K receive buffers (fp32 [ksplit][128 rows][odd number of 16-byte chunks]) reuse the
+    // X ring: the largest over ksplit 2..8
+    static constexpr int recv_bytes(int ks) {
+        return ks * kBlockN * ((((BT + ks - 1) / ks + 3) / 4) | 1) * 16;
+    }
+    static constexpr int max_recv_bytes() {
+        int m = 0;
+        for (int ks = 2; ks <= 8; ++ks) m = recv_bytes(ks) > m ? recv_bytes(ks) : m;
+        return m;
+    }
+    static_assert(PAIR || max_recv_bytes() <= kXStages * kXStageBytes, "split-K receive buffer");
     static constexpr uint32_t kIdesc = idesc_f16_f32(PAIR ? 2 * kBlockN : kBlockN, BT);
 };
 
@@ -621,32 +629,10 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT, PAIR>::kThreads, Cfg<BITS, G
                         *reinterpret_cast<uint32_t*>(p.Y + static_cast<size_t>(m) * p.N + n_pair) = outw;
                 }
             } else {
-                // split-K: this CTA's fp32 partial goes to shared memory, rows of 16-byte chunks
-                // XOR-swizzled by row so that both the writes and the cluster reads are conflict-free
-                float* part = reinterpret_cast<float*>(smem);
-#pragma unroll
-                for (int c0 = 0; c0 < C::kEpiCols; c0 += kChunk) {
-                    uint32_t v[32];
-                    if (kChunk == 32) {
-                        tmem_ld32(lane_base + b * BT + col0 + c0, v);
-                    } else {
-                        tmem_ld16(lane_base + b * BT + col0 + c0, *reinterpret_cast<uint32_t(*)[16]>(v));
-                    }
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int j = 0; j < kChunk; j += 4) {
-                        const int c4 = (col0 + c0 + j) >> 2;
-                        const int pc = c4 ^ (row & C::kPartSwizzle);
-                        *reinterpret_cast<float4*>(part + row * BT + pc * 4) =
-                            make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]), __uint_as_float(v[j + 2]),
-                                        __uint_as_float(v[j + 3]));
-                    }
-                }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&accempty[b]);
-                // The row factors of the tile's tokens, for the reduction below, go to the weight
-                // ring (every stage has been decoded by now): the reduction then reads them from
+                // split-K (one tile per CTA): the accumulator stays in tensor memory until every
+                // rank of the cluster has finished its K slice, when it is pushed to the ranks
+                // that reduce it (below). The row factors of the tile's tokens go to the weight
+                // ring (every stage has been decoded by now), for the reduction to read from
                 // shared memory instead of waiting on a global load behind each store.
                 const int te = (warp - C::kFirstEpiWarp) * 32 + lane;
                 const int mt = (tile / p.n_tiles) * BT;
@@ -657,10 +643,54 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT, PAIR>::kThreads, Cfg<BITS, G
 
     __syncwarp();
     if (split) {
-        // Sum the K-slices of the cluster in rank order. Rank r reduces a contiguous range of the
-        // tile's token columns (multiples of 4), read as 16-byte chunks from every rank.
-        cluster_sync_all();
-        if (warp >= C::kFirstEpiWarp && warp < C::kFirstDqWarp && !*abort_flag) {
+        // Sum the K slices of the cluster in rank order. Rank r owns a contiguous range of the
+        // tile's token columns (a multiple of 4 wide). Once every rank has finished its slice
+        // (barrier 1; their X rings are free), each rank pushes its fp32 partial of every range
+        // into the owner's shared memory with remote stores, which do not wait for a reply;
+        // after barrier 2 every owner adds the ranks' partials from its own shared memory,
+        // scales them by the row factors and stores the bf16 result.
+        // Receive buffer of an owner: [source rank][128 rows][P 16-byte chunks], P = its column
+        // count / 4 made odd, so that 32 rows' chunks at one column fall in distinct banks.
+        const int ks = p.ksplit;
+        const int rank = static_cast<int>(cluster_ctarank());
+        const int per_rank = ((BT + ks - 1) / ks + 3) / 4 * 4;
+        const int chunks = per_rank / 4;
+        const int P = chunks | 1;
+        const uint32_t recv0 = smem_u32(smem);
+        cluster_sync_all();   // barrier 1
+        const bool epi = warp >= C::kFirstEpiWarp && warp < C::kFirstDqWarp;
+        if (epi && !*abort_flag) {
+            tc_fence_after();
+            const int e = warp - C::kFirstEpiWarp;
+            const int quarter = warp & 3;
+            const int row = quarter * 32 + lane;
+            const int col0 = (e >> 2) * C::kEpiCols;
+            const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
+            constexpr int kChunk = (C::kEpiCols >= 32) ? 32 : 16;
+#pragma unroll
+            for (int c0 = 0; c0 < C::kEpiCols; c0 += kChunk) {
+                uint32_t v[32];
+                if (kChunk == 32) {
+                    tmem_ld32(lane_base + col0 + c0, v);
+                } else {
+                    tmem_ld16(lane_base + col0 + c0, *reinterpret_cast<uint32_t(*)[16]>(v));
+                }
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < kChunk; j += 4) {
+                    const int col = col0 + c0 + j;
+                    const int owner = col / per_rank;
+                    const int cl = (col - owner * per_rank) >> 2;
+                    const uint32_t off = static_cast<uint32_t>(((rank * kBlockN + row) * P + cl) * 16);
+                    if (dcheck(owner < ks && off + 16 <= static_cast<uint32_t>(C::kXStages * C::kXStageBytes), status))
+                        st_shared_cluster_v4(map_shared_rank(recv0 + off, static_cast<uint32_t>(owner)),
+                                             make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]),
+                                                         __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3])));
+                }
+            }
+        }
+        cluster_sync_all();   // barrier 2: every push has landed
+        if (epi && !*abort_flag) {
             const int e = warp - C::kFirstEpiWarp;
             const int quarter = warp & 3;
             const int epart = e >> 2;
@@ -668,58 +698,32 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT, PAIR>::kThreads, Cfg<BITS, G
             const int tile = blockIdx.x;
             const int m0 = (tile / p.n_tiles) * BT;
             const int n = (tile % p.n_tiles) * p.rows + row;
-            const int rank = static_cast<int>(cluster_ctarank());
-            const int per_rank = ((BT + p.ksplit - 1) / p.ksplit + 3) / 4 * 4;
             const int cb = rank * per_rank;
-            const int ce = min(BT, cb + per_rank);
-            const uint32_t part0 = smem_u32(smem);
+            const int cend = min(min(BT, cb + per_rank), p.M - m0);
             const float* fac = reinterpret_cast<const float*>(wring);
+            const float4* recv = reinterpret_cast<const float4*>(smem);
             if (row < p.rows && n < p.N) {
-                // kPass 4-column groups per pass (two where registers allow): every rank's
-                // 16-byte chunk of them is requested before any is added, then the ranks are
-                // summed in order and the sums scaled by the row factors staged above and stored.
-                constexpr int kMaxRanks = 8;
-                constexpr int kPass = C::kCtasPerSm == 2 ? 1 : 2;
                 constexpr int kStep = 4 * C::kEpiParts;
-                const int ks = p.ksplit;
-                const int cend = min(ce, p.M - m0);
-                for (int c = cb + 4 * epart; c < cend; c += kPass * kStep) {
-                    float4 v[kPass][kMaxRanks];
-#pragma unroll
-                    for (int h = 0; h < kPass; ++h) {
-                        const int cc = c + h * kStep;
-                        const int pc = (cc >> 2) ^ (row & C::kPartSwizzle);
-                        const uint32_t off = static_cast<uint32_t>((row * BT + pc * 4) * 4);
-#pragma unroll
-                        for (int q = 0; q < kMaxRanks; ++q)
-                            if (q < ks && cc < cend) v[h][q] = ld_shared_cluster_v4(map_shared_rank(part0 + off, q));
+                for (int c = cb + 4 * epart; c < cend; c += kStep) {
+                    const int cl = (c - cb) >> 2;
+                    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                    for (int q = 0; q < ks; ++q) {
+                        const float4 v = recv[(q * kBlockN + row) * P + cl];
+                        acc.x += v.x;
+                        acc.y += v.y;
+                        acc.z += v.z;
+                        acc.w += v.w;
                     }
+                    const float a4[4] = {acc.x, acc.y, acc.z, acc.w};
 #pragma unroll
-                    for (int h = 0; h < kPass; ++h) {
-                        const int cc = c + h * kStep;
-                        if (cc >= cend) break;
-                        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-                        for (int q = 0; q < kMaxRanks; ++q) {
-                            if (q < ks) {
-                                acc.x += v[h][q].x;
-                                acc.y += v[h][q].y;
-                                acc.z += v[h][q].z;
-                                acc.w += v[h][q].w;
-                            }
-                        }
-                        const float a4[4] = {acc.x, acc.y, acc.z, acc.w};
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const int m = m0 + cc + j;
-                            if (m < p.M && dcheck(m >= 0 && n >= 0 && n < p.N && cc + j < BT, status))
-                                p.Y[static_cast<size_t>(m) * p.N + n] = __float2bfloat16_rn(a4[j] * fac[cc + j]);
-                        }
+                    for (int j = 0; j < 4; ++j) {
+                        const int m = m0 + c + j;
+                        if (m < p.M && dcheck(m >= 0 && n >= 0 && n < p.N && c + j < BT, status))
+                            p.Y[static_cast<size_t>(m) * p.N + n] = __float2bfloat16_rn(a4[j] * fac[c + j]);
                     }
                 }
             }
         }
-        cluster_sync_all();
     }
 
     tc_fence_before();
