@@ -94,7 +94,11 @@ def is_hbm_bound(flops: float, nbytes: float, peaks: dict) -> bool:
     return flops / nbytes < ridge
 
 
-def measure_shapes(items, copies, lb, torch, device, stream, cap_stream, samples=9, replays=5):
+SHAPE_SAMPLES, SHAPE_REPLAYS = 21, 4   # per-launch timing: median of 21 samples of 4 graph replays
+
+
+def measure_shapes(items, copies, lb, torch, device, stream, cap_stream, samples=SHAPE_SAMPLES,
+                   replays=SHAPE_REPLAYS):
     """Per-launch durations of each distinct shape of `items` (ms): {(M, K, N): (call, GEMM kernel,
     X conversion, reps)}.
 
@@ -219,7 +223,7 @@ def measure_step_config(name, lb, torch, device, stream, cap_stream, peaks, l2_b
 
 def measure_configs(lb, torch, device, stream, cap_stream, peaks, l2_bytes):
     """Per-launch results of the reference configurations (see CONFIGS), each linear timed as in
-    measure_shapes with fewer samples: per shape the call, GEMM kernel and conversion times, the
+    measure_shapes with fewer replays per sample: per shape the call, GEMM kernel and conversion times, the
     throughput of the GEMM kernel and its fraction of the burst bf16 peak (tensor-bound) or of the
     HBM bandwidth (HBM-bound)."""
     out = {}
@@ -227,7 +231,7 @@ def measure_configs(lb, torch, device, stream, cap_stream, peaks, l2_bytes):
         specs = synth.WORKLOADS[name]
         copies = rotation_copies(step_bytes(specs), weight_bytes(specs), l2_bytes)
         items, _ = setup(specs, device, lb, torch, pinned=False, copies=copies)
-        times = measure_shapes(items, copies, lb, torch, device, stream, cap_stream, samples=5, replays=3)
+        times = measure_shapes(items, copies, lb, torch, device, stream, cap_stream, samples=21, replays=2)
         hbm = is_hbm_bound(step_flops(specs), step_bytes(specs), peaks)
         shapes = []
         for sp in specs:
@@ -541,7 +545,8 @@ def run_lowbit(args, specs, workload):
     conv_ms = sum(v for _, _, _, v in per) / len(per)
     launch_flops = sum(sp.flops for sp, _, _, _ in per) / len(per)
     launch_bytes = sum(sp.algorithmic_bytes() for sp, _, _, _ in per) / len(per)
-    launches_timed = sum(2 * 9 * 5 * r if k[0] > 16 else 9 * 5 * r for k, (_, _, _, r) in shape_times.items())
+    per_graph = SHAPE_SAMPLES * SHAPE_REPLAYS
+    launches_timed = sum((2 if k[0] > 16 else 1) * per_graph * r for k, (_, _, _, r) in shape_times.items())
     # Per-launch figures of the other reference configurations, measured the same way after the
     # headline's timed region (so that one run of the default workload corroborates them).
     others = None
