@@ -223,7 +223,7 @@ template <int BITS, int GS, int BT, bool PAIR>
 __global__ void __launch_bounds__(Cfg<BITS, GS, BT, PAIR>::kThreads, Cfg<BITS, GS, BT, PAIR>::kCtasPerSm)
     lowbit_gemm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w,
                        const __grid_constant__ CUtensorMap map_s, const __grid_constant__ CUtensorMap map_z,
-                       const KernelParams p) {
+                       const __grid_constant__ CUtensorMap map_y, const KernelParams p) {
     using C = Cfg<BITS, GS, BT, PAIR>;
     constexpr int SX = C::kXStages;
     constexpr int SW = C::kWStages;
@@ -282,6 +282,7 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT, PAIR>::kThreads, Cfg<BITS, G
         tma_prefetch_desc(&map_w);
         tma_prefetch_desc(&map_s);
         if (BITS == 4) tma_prefetch_desc(&map_z);
+        tma_prefetch_desc(&map_y);
     }
     if (warp == 1) {
         tmem_alloc<PAIR>(tmem_holder, C::kTmemCols);
@@ -582,7 +583,58 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT, PAIR>::kThreads, Cfg<BITS, G
             }
             if (!__all_sync(0xffffffffu, mbar_wait(&accfull[b], acc_ph, abort_flag, status))) break;
             tc_fence_after();
-            if (!split) {
+            if (!split && t + 1 == my_tiles) {
+                // The CTA's last tile has nothing to overlap its stores with, and its X ring is
+                // idle (the MMAs just completed consumed every stage): the tile goes, chunk by
+                // chunk, to X stage 0 as the Y box [BT tokens][p.rows rows] and leaves in one TMA
+                // store, which clips the parts past M or N.
+                uint32_t* stg = reinterpret_cast<uint32_t*>(smem);
+                const bool even = (lane & 1) == 0;
+                const int r_pair = row - (even ? 0 : 1);   // the pair's even row within the tile
+#pragma unroll 1
+                for (int c0 = 0; c0 < C::kEpiCols; c0 += kChunk) {
+                    uint32_t v[32];
+                    if (kChunk == 32) {
+                        tmem_ld32(lane_base + b * BT + col0 + c0, v);
+                    } else {
+                        tmem_ld16(lane_base + b * BT + col0 + c0, *reinterpret_cast<uint32_t(*)[16]>(v));
+                    }
+                    float mul_j = mul[0];
+#pragma unroll
+                    for (int ci = 1; ci < kChunks; ++ci)
+                        if (ci == c0 / kChunk) mul_j = mul[ci];   // keeps mul[] in registers
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < kChunk; j += 2) {
+                        const float f0 = __uint_as_float(v[j]) * __shfl_sync(0xffffffffu, mul_j, j);
+                        const float f1 = __uint_as_float(v[j + 1]) * __shfl_sync(0xffffffffu, mul_j, j + 1);
+                        const __nv_bfloat162 h2 = __floats2bfloat162_rn(f0, f1);   // (token j, token j+1)
+                        const uint32_t mine = *reinterpret_cast<const uint32_t*>(&h2);
+                        // lanes 2i, 2i+1 (rows n, n+1) swap halves: (row n, row n+1) at one token
+                        const uint32_t other = __shfl_xor_sync(0xffffffffu, mine, 1);
+                        const uint32_t outw =
+                            even ? __byte_perm(mine, other, 0x5410) : __byte_perm(other, mine, 0x7632);
+                        const int ml = col0 + c0 + j + (even ? 0 : 1);   // token within the tile
+                        if (r_pair < p.rows && dcheck((ml * p.rows + r_pair) * 2 + 4 <= C::kXStageBytes, status))
+                            stg[(ml * p.rows + r_pair) >> 1] = outw;
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    if (PAIR && !issuer)
+                        mbar_arrive_remote(on_issuer(&accempty[b]));
+                    else
+                        mbar_arrive(&accempty[b]);
+                }
+                fence_proxy_async_smem();
+                named_bar_sync(1, 32 * C::kNumEpiWarps);
+                if (e == 0 && lane == 0) {
+                    tma_store_2d(&map_y, smem, (tile % p.n_tiles) * n_stride + n_off, (tile / p.n_tiles) * BT);
+                    bulk_commit_group();
+                    bulk_wait_read_all();   // the shared memory may not be released before this
+                }
+            } else if (!split) {
                 // Read the whole slice into registers (scaled, rounded to bf16), hand the
                 // accumulator back to the MMA issuer, then store: the stores of this tile
                 // overlap the next tile's MMAs.
@@ -1080,6 +1132,10 @@ lowbit_status launch(const GemmProblem& g, int rows, int ksplit_request, cudaStr
                                kBlockN, C::kGroupsPerStage, CU_TENSOR_MAP_SWIZZLE_NONE);
     else
         mz = ms;
+    // Y as (N, M) with a box of one tile, [BT tokens][rows]: the store of each CTA's last tile
+    CUtensorMap my;
+    ok = ok && make_map_2d(&my, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.Y, N, M, uint64_t(N) * 2, rows, BT,
+                           CU_TENSOR_MAP_SWIZZLE_NONE);
     if (!ok) return LOWBIT_ERR_CUDA;
 
     KernelParams p;
@@ -1161,7 +1217,7 @@ lowbit_status launch(const GemmProblem& g, int rows, int ksplit_request, cudaStr
     cfg.attrs = attrs;
     cfg.numAttrs = na;
     if (take_injected_failure(kInjectLaunch)) return LOWBIT_ERR_CUDA;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, mx, mw, ms, mz, p);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, mx, mw, ms, mz, my, p);
     return e == cudaSuccess ? LOWBIT_OK : LOWBIT_ERR_CUDA;
 }
 
