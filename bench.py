@@ -41,7 +41,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # The sources each kernel is built from (besides the headers every kernel includes): a capture
 # stays valid while these are unchanged.
-KERNEL_SOURCES = {"lowbit_gemm_kernel": ("gemm_sm100.cu",),
+KERNEL_SOURCES = {"lowbit_gemm_kernel": ("gemm_sm100.cu", "tcgen05_ptx.cuh"),
                   "lowbit_smallm_kernel": ("smallm_kernel.cuh", "smallm_host.cu", "smallm_b1.cu", "smallm_b2.cu",
                                            "smallm_b4.cu")}
 SHARED_SOURCES = ("sm100_ptx.cuh", "lowbit_internal.h")

@@ -53,6 +53,7 @@
 
 #include "lowbit_internal.h"
 #include "sm100_ptx.cuh"
+#include "tcgen05_ptx.cuh"
 
 namespace lowbit {
 

@@ -164,12 +164,6 @@ __device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t* p, uint32_t v) {
 }
 
 
-__device__ __forceinline__ void st_shared_cluster_v4(uint32_t addr, float4 v) {
-    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.x), "f"(v.y), "f"(v.z),
-                 "f"(v.w)
-                 : "memory");
-}
-
 // Exact bf16 pairs of two neighbouring codes (k, k + 1) at pair index c of a packed word (c a
 // compile-time constant after unrolling, so pair 0 needs no shift).
 __device__ __forceinline__ uint32_t dec_u4(uint32_t v, int c) {       // 128 + q
