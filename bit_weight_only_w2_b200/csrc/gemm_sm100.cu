@@ -141,6 +141,9 @@ struct Cfg {
     }
     static_assert(PAIR || max_recv_bytes() <= kXStages * kXStageBytes, "split-K receive buffer");
     static constexpr uint32_t kIdesc = idesc_f16_f32(PAIR ? 2 * kBlockN : kBlockN, BT);
+    // the last tile's bf16 Y box [BT][128 rows] is staged at the start of the (idle) X ring
+    static constexpr int kYStageBytes = BT * kBlockN * 2;
+    static_assert(kYStageBytes <= kXStages * kXStageBytes, "Y staging");
 };
 
 struct KernelParams {
@@ -586,9 +589,10 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT, PAIR>::kThreads, Cfg<BITS, G
             tc_fence_after();
             if (!split && t + 1 == my_tiles) {
                 // The CTA's last tile has nothing to overlap its stores with, and its X ring is
-                // idle (the MMAs just completed consumed every stage): the tile goes, chunk by
-                // chunk, to X stage 0 as the Y box [BT tokens][p.rows rows] and leaves in one TMA
-                // store, which clips the parts past M or N.
+                // idle (the MMAs just completed consumed every stage, and no copy is in flight):
+                // the tile goes, chunk by chunk, to the start of the X ring as the Y box [BT
+                // tokens][p.rows rows] (one X stage, or two of a CTA pair's half-size stages) and
+                // leaves in one TMA store, which clips the parts past M or N.
                 uint32_t* stg = reinterpret_cast<uint32_t*>(smem);
                 const bool even = (lane & 1) == 0;
                 const int r_pair = row - (even ? 0 : 1);   // the pair's even row within the tile
@@ -616,7 +620,7 @@ __global__ void __launch_bounds__(Cfg<BITS, GS, BT, PAIR>::kThreads, Cfg<BITS, G
                         const uint32_t outw =
                             even ? __byte_perm(mine, other, 0x5410) : __byte_perm(other, mine, 0x7632);
                         const int ml = col0 + c0 + j + (even ? 0 : 1);   // token within the tile
-                        if (r_pair < p.rows && dcheck((ml * p.rows + r_pair) * 2 + 4 <= C::kXStageBytes, status))
+                        if (r_pair < p.rows && dcheck((ml * p.rows + r_pair) * 2 + 4 <= C::kYStageBytes, status))
                             stg[(ml * p.rows + r_pair) >> 1] = outw;
                     }
                 }

@@ -96,3 +96,37 @@ def test_debug_build_index_checks():
     assert dbg.lowbit_selftest_index_check(stream) == 0
     assert dbg.lowbit_last_device_status(stream) == LOWBIT_ERR_DEVICE_CHECK
     assert dbg.lowbit_last_device_status(stream) == 0
+
+
+# (bits, gs, M, K, N, tile_tokens, tile_rows, ksplit): CTA-pair tiles (several per pair, and a
+# ragged token tile), K split 2, 3 and 7 ways (the push reduction), flat row tiles, 16- to
+# 128-token tiles, and single-tile launches (the last tile's TMA store) with ragged N.
+DEBUG_CASES = [(2, 128, 2304, 256, 2560, 0, 256, 0), (4, 64, 300, 384, 768, 0, 256, 0),
+               (1, 128, 300, 1024, 512, 0, 256, 0), (2, 128, 512, 3072, 264, 256, 128, 2),
+               (4, 64, 200, 768, 264, 256, 0, 3), (2, 64, 300, 1792, 520, 128, 0, 7),
+               (2, 128, 40, 768, 264, 32, 72, 1), (1, 64, 70, 1024, 136, 16, 0, 0), (4, 128, 129, 512, 1032, 0, 0, 0)]
+
+
+@pytest.mark.parametrize("case", DEBUG_CASES, ids=lambda c: "b{}g{}_{}x{}x{}_bt{}_rows{}_ks{}".format(*c))
+def test_debug_build_checks_every_tile_path(case):
+    """The debug build's index checks stay silent on the CTA-pair, split-K (push reduction), flat
+    and staged-store paths, and its results equal the release build's and match the oracle."""
+    bits_, gs, M, K, N, bt, rows, ks = case
+    spec = spec_for(bits_, gs, M, K, N, seed=sum(case))
+    prob = synth.make_problem(spec)
+    x, packed, s, z = _gpu.dev_problem(prob)
+    ws = torch.empty(lb.workspace_size(M, K), dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream().cuda_stream
+    outs = []
+    for lib in (lb.load(), lb.load_debug()):
+        y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+        st = lib.lowbit_gemm_ex(M, N, K, bits_, gs, x.data_ptr(), packed.data_ptr(), s.data_ptr(),
+                                None if z is None else z.data_ptr(), y.data_ptr(), ws.data_ptr(), ws.numel(), bt,
+                                rows, ks, stream)
+        assert st == 0
+        torch.cuda.synchronize()
+        assert lib.lowbit_last_device_status(stream) == 0, spec.name
+        outs.append(y)
+    assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16)), spec.name
+    ref = oracle.gemm(prob.x_bf16, _gpu.oracle_packed(prob), prob.scales, prob.zeros, N, bits_, gs)
+    _gpu.check_close(_gpu.y_to_f64(outs[1]), ref, what=spec.name)
