@@ -195,6 +195,10 @@ WORKLOADS = {
     # four text-encoder MLP layers (gate, up, down) at 512 and at 16 tokens
     "te_mlp4_m512_uint4_g64": text_encoder_mlp_layers(512),
     "te_mlp4_m16_uint4_g64": text_encoder_mlp_layers(16),
+    # the small-M kernel's sustained rate: one uint4 linear at 16 tokens with a K long enough
+    # (40 steps of 512) that start-up is amortized; not a model shape
+    "smallm_steady_m16_uint4_g64": [LinearSpec("steady16", 16, 20480, 9472, bits=4, group_size=64,
+                                               scale_lo=0.002, scale_hi=0.01)],
     # the transformer's ternary and binary linear shapes at 1, 4 and 16 tokens (HBM-bound)
     **{f"klein_linears_m{m}_{'ternary' if b == 2 else 'binary'}_g128": klein_linears_small_m(m, b)
        for b in (2, 1) for m in (1, 4, 16)},

@@ -318,7 +318,7 @@ def sampled_check(spec, seed=0, n_random=4096, n_rows=16, n_cols=16):
     return _gpu.check_close(y[ms, ns], ref, rms=rms, what=spec.name)
 
 
-FULL_WHOLE = [s for w in ("qkv_512sq_ternary_g128", "te_m512_uint4_g64", "te_m16_uint4_g64",
+FULL_WHOLE = [s for w in ("qkv_512sq_ternary_g128", "te_m512_uint4_g64", "te_m16_uint4_g64", "smallm_steady_m16_uint4_g64",
                            *(f"klein_linears_m{m}_{f}_g128" for f in ("ternary", "binary") for m in (1, 4, 16)))
               for s in synth.WORKLOADS[w]]
 FULL_SAMPLED = synth.WORKLOADS["mlp_1024sq_binary_g128"]
