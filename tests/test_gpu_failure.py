@@ -100,17 +100,23 @@ def test_debug_build_index_checks():
 
 # (bits, gs, M, K, N, tile_tokens, tile_rows, ksplit): CTA-pair tiles (several per pair, and a
 # ragged token tile), K split 2, 3 and 7 ways (the push reduction), flat row tiles, 16- to
-# 128-token tiles, and single-tile launches (the last tile's TMA store) with ragged N.
+# 128-token tiles, single-tile launches (the last tile's TMA store) with ragged N, and the
+# small-M kernel in both orientations.
 DEBUG_CASES = [(2, 128, 2304, 256, 2560, 0, 256, 0), (4, 64, 300, 384, 768, 0, 256, 0),
                (1, 128, 300, 1024, 512, 0, 256, 0), (2, 128, 512, 3072, 264, 256, 128, 2),
                (4, 64, 200, 768, 264, 256, 0, 3), (2, 64, 300, 1792, 520, 128, 0, 7),
-               (2, 128, 40, 768, 264, 32, 72, 1), (1, 64, 70, 1024, 136, 16, 0, 0), (4, 128, 129, 512, 1032, 0, 0, 0)]
+               (2, 128, 40, 768, 264, 32, 72, 1), (1, 64, 70, 1024, 136, 16, 0, 0), (4, 128, 129, 512, 1032, 0, 0, 0),
+               # the small-M kernel: X as the 16-row operand (automatic tiles, a forced 3-way split
+               # with ragged N) and weights as the 16-row operand (split 2)
+               (4, 64, 16, 2560, 9728, 1, 0, 0), (4, 64, 16, 9728, 2560, 1, 0, 0), (1, 128, 12, 1536, 1032, 1, 48, 3),
+               (2, 128, 5, 3072, 264, 8, 16, 2), (4, 64, 3, 2048, 520, 8, 0, 0)]
 
 
 @pytest.mark.parametrize("case", DEBUG_CASES, ids=lambda c: "b{}g{}_{}x{}x{}_bt{}_rows{}_ks{}".format(*c))
 def test_debug_build_checks_every_tile_path(case):
-    """The debug build's index checks stay silent on the CTA-pair, split-K (push reduction), flat
-    and staged-store paths, and its results equal the release build's and match the oracle."""
+    """The debug build's index checks stay silent on the CTA-pair, split-K (push reduction), flat,
+    staged-store and small-M paths, and its results equal the release build's and match the
+    oracle."""
     bits_, gs, M, K, N, bt, rows, ks = case
     spec = spec_for(bits_, gs, M, K, N, seed=sum(case))
     prob = synth.make_problem(spec)
