@@ -537,3 +537,39 @@ def test_small_m_row_magnitudes(bits, gs, M, tile_tokens):
         if m == 2:
             continue
         _gpu.check_close(y[m:m + 1], ref[m:m + 1], what=f"row {m}")
+
+
+def test_concurrent_host_threads_match_sequential_calls():
+    """Four host threads, each with its own stream and workspace, run linears of every kernel
+    path at once (the binding releases the GIL in the C calls): the library's host caches --
+    tensor maps, cluster capacities, shared-memory opt-ins -- are shared by the threads, and every
+    output equals the sequential call's bit for bit."""
+    from concurrent.futures import ThreadPoolExecutor
+    shapes = [(2, 128, 2304, 256, 2560), (4, 64, 16, 2560, 1032), (1, 128, 300, 1024, 520), (4, 64, 200, 768, 264),
+              (2, 128, 5, 3072, 264), (2, 64, 40, 768, 264), (1, 64, 513, 512, 768), (4, 128, 1024, 512, 1024)]
+    items = []
+    for i, (b, g, m, k, n) in enumerate(shapes):
+        sp = spec_for(b, g, m, k, n, seed=900 + i)
+        items.append((sp, _gpu.dev_problem(synth.make_problem(sp))))
+    want = [lb.gemm(x, w, s, z, sp.bits, sp.group_size) for sp, (x, w, s, z) in items]
+    torch.cuda.synchronize()
+
+    def worker(t):
+        stream = torch.cuda.Stream()
+        ws = torch.empty(max(lb.workspace_size(sp.M, sp.K) for sp, _ in items), dtype=torch.uint8, device="cuda")
+        outs = []
+        with torch.cuda.stream(stream):
+            for r in range(3):
+                for j in range(len(items)):
+                    sp, (x, w, s, z) = items[(j + t) % len(items)]
+                    outs.append(((j + t) % len(items), lb.gemm(x, w, s, z, sp.bits, sp.group_size, ws=ws)))
+        stream.synchronize()
+        return outs
+
+    with ThreadPoolExecutor(4) as pool:
+        results = list(pool.map(worker, range(4)))
+    torch.cuda.synchronize()
+    assert lb.device_status() == 0
+    for outs in results:
+        for j, y in outs:
+            assert torch.equal(y.view(torch.int16), want[j].view(torch.int16)), items[j][0].name
