@@ -220,3 +220,29 @@ def test_binding_rejects_cpu_tensors_and_bad_descs():
         lb.make_desc(x, packed, s, z, torch.zeros((16, 64), dtype=torch.bfloat16), 2, 128)
     with pytest.raises(ValueError, match="packed: 8 words"):
         lb.unpack(torch.zeros((2, 4), dtype=torch.int32), 4, 64, 2)
+
+
+def test_binding_without_the_library_raises(tmp_path):
+    """A copy of the Python package with no built library refuses to load instead of running
+    anything else: the product path has no CPU fallback."""
+    import shutil
+    import subprocess
+    import sys
+    pkg = os.path.join(ROOT, "bit_weight_only_w2_b200")
+    dst = tmp_path / "bit_weight_only_w2_b200"
+    dst.mkdir()
+    for f in os.listdir(pkg):
+        if f.endswith(".py"):
+            shutil.copy(os.path.join(pkg, f), dst / f)
+    code = ("import bit_weight_only_w2_b200 as lb, sys\n"
+            "assert lb.__file__.startswith(sys.argv[1]), lb.__file__\n"
+            "try:\n"
+            "    lb.load()\n"
+            "except FileNotFoundError as e:\n"
+            "    print('raised', e)\n"
+            "else:\n"
+            "    raise SystemExit('loaded without a library')\n")
+    r = subprocess.run([sys.executable, "-c", code, str(tmp_path)], cwd=str(tmp_path), capture_output=True,
+                       text=True, timeout=300, env={**os.environ, "PYTHONPATH": str(tmp_path)})
+    assert r.returncode == 0, r.stderr + r.stdout
+    assert "raised" in r.stdout and "liblowbit.so is missing" in r.stdout
