@@ -34,7 +34,7 @@
 //   * eight warps, each taking 64 of the step's 512 K (one group or half of one) for all the
 //     tile's octets (kHalves = 2 instead runs sixteen warps of 128 registers, warps w and w + 8
 //     sharing a K chunk with half the octets each). A warp turns its group's fp16 scales /
-//     zeros for its rows into fp32 pairs (s, s * c), loads its four X fragments once with
+//     zeros for its rows into fp32 pairs (s, -s * c), loads its four X fragments once with
 //     ldmatrix, forms Sx with four MMAs against ones, and runs the decode + MMA chains of its
 //     octets, each lane loading one 32-bit code word per block of block-ordered codes;
 //   * at the end of a tile the eight K-chunk partial sums of every octet are added in a fixed
@@ -111,7 +111,7 @@ bool layout(int rows, int ksplit, bool swap, Params* p, int* smem_bytes) {
     const uint32_t end = p->z_off + (BITS == 4 ? s_bytes : 0);
     p->stage_bytes = (end + 1023) / 1024 * 1024;
     p->tx_bytes = xb + w_bytes + s_raw * (BITS == 4 ? 2 : 1);
-    // per warp, fp32 (s, s * c) of its rows: four float4 per octet (pairs of rows), or eight per
+    // per warp, fp32 (s, -s * c) of its rows: four float4 per octet (pairs of rows), or eight per
     // unit with `swap` (rows g and g + 8 of the unit for each g)
     const uint32_t scr = kWarps * (swap ? 8 : 4) * ((units + kHalves - 1) / kHalves) * 16;
     const uint32_t red = 4 * units * 512;
@@ -154,6 +154,15 @@ __device__ __forceinline__ void mma_bf16_z(float (&d)[4], const uint32_t (&a)[4]
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.f));
 }
 
+// (d0, d1) = (a0 * b0 + d0, a1 * b1 + d1): one packed fp32 FMA (each lane rounded once, as fmaf).
+__device__ __forceinline__ void fma_f32x2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+    asm("{\n\t.reg .b64 rd, ra, rb;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rd, {%0, %1};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rd;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "+f"(d0), "+f"(d1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
 __device__ __forceinline__ void cta_bar() { asm volatile("bar.sync 1, %0;" ::"n"(kThreads) : "memory"); }
 
 // Shared-memory counter increment with acquire-release ordering at CTA scope; returns the old value.
@@ -184,7 +193,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     using F = Fmt<BITS, GS>;
     static_assert(!SWAP || NOCT % 2 == 0, "weights as the 16-row operand take rows in pairs of octets");
     constexpr int R = 8 * NOCT;                       // weight rows per tile
-    constexpr int HALF = R / 2;                       // (s, s * c) pairs per group
     constexpr int NUT = SWAP ? NOCT / 2 : NOCT;       // MMA units per tile: octets, or 16-row pairs of octets
     constexpr int NH = (NUT + kHalves - 1) / kHalves; // units per warp (its half of the tile)
     constexpr int HP = (SWAP ? 8 : 4) * NH;           // scale-table entries of a warp
@@ -310,13 +318,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int o = 0; o < NH; ++o) acc[o][0] = acc[o][1] = acc[o][2] = acc[o][3] = 0.f;
 
     // ---- the phases of one ring step, shared by both loop drivers below ----
-    // P1: this warp's group: fp32 (s, s * c) of every row of its units, into `tab`
+    // P1: this warp's group: fp32 (s, -s * c) of every row of its units, into `tab` (negated so
+    // that the scale epilogue is two packed FMAs per pair of accumulators)
     auto build_table = [&](const uint8_t* st, float4* tab) {
         const __half* sh = reinterpret_cast<const __half*>(st + p.s_off) + gi * R;
         const __half* zh = reinterpret_cast<const __half*>(st + p.z_off) + gi * R;
         auto sc_of = [&](int r, float& sf, float& cf) {
             sf = __half2float(sh[r]);
-            cf = BITS == 4 ? sf * (128.f + __half2float(zh[r])) : BITS == 2 ? 129.f * sf : 0.f;
+            cf = BITS == 4 ? -(sf * (128.f + __half2float(zh[r]))) : BITS == 2 ? -(129.f * sf) : 0.f;
         };
         if constexpr (SWAP) {
             // entry 8u + g: rows 16u + g and 16u + g + 8 of the warp's units
@@ -342,11 +351,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     float c0 = 0.f, c1 = 0.f;
                     if (BITS == 4) {
                         const float2 zf = __half22float2(zp[i]);
-                        c0 = sf.x * (128.f + zf.x);
-                        c1 = sf.y * (128.f + zf.y);
+                        c0 = -(sf.x * (128.f + zf.x));
+                        c1 = -(sf.y * (128.f + zf.y));
                     } else if (BITS == 2) {
-                        c0 = 129.f * sf.x;
-                        c1 = 129.f * sf.y;
+                        c0 = -(129.f * sf.x);
+                        c1 = -(129.f * sf.y);
                     }
                     tab[i] = make_float4(sf.x, sf.y, c0, c1);
                 }
@@ -445,7 +454,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     };
-    // P6: scale the group sums and add them to the accumulators
+    // P6: scale the group sums and add them to the accumulators, acc += s * T + (-s * c) * Sx, as
+    // packed fp32 FMAs over pairs of accumulators (bit-identical to one fmaf per element)
     auto scale_units = [&](const float (&T)[B][4], const float (&tsx)[4], const float4* tab, int ob) {
 #pragma unroll
         for (int u = 0; u < B; ++u) {
@@ -454,28 +464,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if constexpr (SWAP) {
                     // d: (row g, token 2q), (row g, 2q + 1), (row g + 8, 2q), (row g + 8, 2q + 1)
                     const float4 sc = tab[8 * (ob + u) + g];
-                    d[0] = fmaf(sc.x, T[u][0], d[0]);
-                    d[1] = fmaf(sc.x, T[u][1], d[1]);
-                    d[2] = fmaf(sc.y, T[u][2], d[2]);
-                    d[3] = fmaf(sc.y, T[u][3], d[3]);
+                    fma_f32x2(d[0], d[1], sc.x, sc.x, T[u][0], T[u][1]);
+                    fma_f32x2(d[2], d[3], sc.y, sc.y, T[u][2], T[u][3]);
                     if (BITS != 1) {
-                        d[0] = fmaf(-sc.z, tsx[0], d[0]);
-                        d[1] = fmaf(-sc.z, tsx[1], d[1]);
-                        d[2] = fmaf(-sc.w, tsx[0], d[2]);
-                        d[3] = fmaf(-sc.w, tsx[1], d[3]);
+                        fma_f32x2(d[0], d[1], sc.z, sc.z, tsx[0], tsx[1]);
+                        fma_f32x2(d[2], d[3], sc.w, sc.w, tsx[0], tsx[1]);
                     }
                 } else {
                     // d: (token g, row 2q), (g, 2q + 1), (g + 8, 2q), (g + 8, 2q + 1)
                     const float4 sc = tab[4 * (ob + u) + q];
-                    d[0] = fmaf(sc.x, T[u][0], d[0]);
-                    d[1] = fmaf(sc.y, T[u][1], d[1]);
-                    d[2] = fmaf(sc.x, T[u][2], d[2]);
-                    d[3] = fmaf(sc.y, T[u][3], d[3]);
+                    fma_f32x2(d[0], d[1], sc.x, sc.y, T[u][0], T[u][1]);
+                    fma_f32x2(d[2], d[3], sc.x, sc.y, T[u][2], T[u][3]);
                     if (BITS != 1) {
-                        d[0] = fmaf(-sc.z, tsx[0], d[0]);
-                        d[1] = fmaf(-sc.w, tsx[0], d[1]);
-                        d[2] = fmaf(-sc.z, tsx[2], d[2]);
-                        d[3] = fmaf(-sc.w, tsx[2], d[3]);
+                        fma_f32x2(d[0], d[1], sc.z, sc.w, tsx[0], tsx[0]);
+                        fma_f32x2(d[2], d[3], sc.z, sc.w, tsx[2], tsx[2]);
                     }
                 }
             }
