@@ -197,6 +197,22 @@ def pin_decode_closed_forms(orc):
     assert np.array_equal(W, codes.astype(np.float64) * s_full)
 
 
+def pin_decode_invalid_ternary_field(orc):
+    # reading r2: ternary field 3 is not a code, so it must never decode to a finite weight; it
+    # poisons exactly the weights it occupies (and the outputs that use them), nothing else
+    N, K, g = 2, 64, 64
+    p, _ = orc.pack(np.zeros((N, K), dtype=np.int8), 2)       # all fields 1 (t = 0)
+    p[1, 1] = 0xFFFFFFFF                                        # row 1: one word of fields 3
+    s = f16(np.full((1, N), 0.5))
+    W = orc.decode(p, s, None, N, K, 2, g)
+    bad = np.isnan(W)
+    assert bad[1].sum() == 16 and not bad[0].any(), "exactly the 16 fields of the word are poisoned"
+    assert np.array_equal(W[~bad], np.zeros(int((~bad).sum())))
+    x = bf16_bits_from_f32(np.ones((1, K)))
+    y = orc.gemm(x, p, s, None, N, 2, g)
+    assert y[0, 0] == 0.0 and np.isnan(y[0, 1])
+
+
 def pin_decode_one_hot(orc):
     N, K, g = 20, 128, 64
     G = K // g

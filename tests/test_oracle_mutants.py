@@ -39,6 +39,8 @@ MUTATIONS = {
                                     "return 4 * cpw * b + 8 * q + 2 * p + d;"),
     "block_order_not_used": ("if (bits != 1 && j < wpr / 4 * 4) {", "if (bits != 1 && j < 0) {"),
     "unpack_lane_from_pair_index": ("*j = 4 * b + (r % 8) / 2;", "*j = 4 * b + (r / 8) % 4;"),
+    "invalid_ternary_field_decodes_zero": ("if (f == 3) return NAN;", "if (f == 3) return 0.0;"),
+    "invalid_ternary_field_not_checked": ("if (f == 3) return NAN;", "if (f == 4) return NAN;"),
     "ternary_field_map": ("if (c >= -1 && c <= 1) { *field = (uint32_t)(c + 1); return 0; }",
                           "if (c >= -1 && c <= 1) { *field = (uint32_t)(c + 1) ^ 2u; return 0; }"),
 }
